@@ -1,0 +1,195 @@
+"""Pins for the oracle's paged append and ragged attention: brute-force dense
+attention (torch SDPA in float64 with an explicit mask), closed forms (uniform
+keys, single admitted key), and invariants (block permutation, chunking,
+window >= length, grouped-query replication)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import (PagedCache, append_kv, attend_contiguous, bf16_bits_to_f64,
+                    ragged_attention, token_positions)
+from oracle.forward import splitfuse_pass
+from ragged_paged_kv_b200 import workloads as W
+from ragged_paged_kv_b200.workloads import f32_to_bf16_bits
+
+
+def _bits(rng, shape):
+    return f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
+
+
+def _sdpa_reference(q_lens, ctx_lens, Kc, Vc, Q, Hq, Hkv, window, scale):
+    """Dense per-sequence attention with an explicit L x L boolean mask,
+    float64, through torch's scaled_dot_product_attention."""
+    out = []
+    start = 0
+    g = Hq // Hkv
+    for s, (qs, cs) in enumerate(zip(q_lens, ctx_lens)):
+        L = cs + qs
+        qpos = torch.arange(cs, L)
+        kpos = torch.arange(L)
+        mask = kpos[None, :] <= qpos[:, None]
+        if window > 0:
+            mask &= kpos[None, :] > qpos[:, None] - window
+        q = torch.from_numpy(bf16_bits_to_f64(Q[start:start + qs])).permute(1, 0, 2)    # [Hq, qs, d]
+        k = torch.from_numpy(bf16_bits_to_f64(Kc[s][:L])).permute(1, 0, 2).repeat_interleave(g, 0)
+        v = torch.from_numpy(bf16_bits_to_f64(Vc[s][:L])).permute(1, 0, 2).repeat_interleave(g, 0)
+        o = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None],
+                                                             attn_mask=mask[None, None], scale=scale)
+        out.append(o[0].permute(1, 0, 2).numpy())
+        start += qs
+    return np.concatenate(out, axis=0)
+
+
+@pytest.mark.parametrize("d,Hq,Hkv,window", [(16, 2, 2, 0), (64, 4, 4, 0), (64, 4, 2, 0),
+                                             (16, 4, 1, 5), (64, 2, 2, 1)])
+def test_brute_force_dense_attention(d, Hq, Hkv, window):
+    rng = np.random.default_rng(d * 100 + Hq * 10 + Hkv + window)
+    q_lens, ctx_lens = [9, 1, 1, 20], [0, 37, 5, 44]
+    B, nblk = 16, 32
+    perm = rng.permutation(nblk)
+    bt = np.full((4, 4), -1, np.int32)
+    o = 0
+    for s in range(4):
+        n = -(-(q_lens[s] + ctx_lens[s]) // B)
+        bt[s, :n] = perm[o:o + n]
+        o += n
+    cache = PagedCache(nblk, Hkv, B, d)
+    Kc = [_bits(rng, (q + c, Hkv, d)) for q, c in zip(q_lens, ctx_lens)]
+    Vc = [_bits(rng, (q + c, Hkv, d)) for q, c in zip(q_lens, ctx_lens)]
+    for s in range(4):
+        cache.write_positions(bt[s], np.arange(ctx_lens[s]), Kc[s][:ctx_lens[s]], Vc[s][:ctx_lens[s]])
+    k_new = np.concatenate([Kc[s][ctx_lens[s]:] for s in range(4)])
+    v_new = np.concatenate([Vc[s][ctx_lens[s]:] for s in range(4)])
+    append_kv(cache, bt, q_lens, ctx_lens, k_new, v_new)
+    T = sum(q_lens)
+    Q = _bits(rng, (T, Hq, d))
+    scale = 1 / np.sqrt(d)
+    ours = ragged_attention(cache, bt, q_lens, ctx_lens, Q, scale, window)
+    ref = _sdpa_reference(q_lens, ctx_lens, Kc, Vc, Q, Hq, Hkv, window, scale)
+    assert np.abs(ours - ref).max() <= 1e-12
+
+
+def test_append_is_a_bit_copy_and_leaves_other_slots():
+    rng = np.random.default_rng(1)
+    q_lens, ctx_lens = np.array([5, 1, 17]), np.array([0, 33, 14])
+    B, Hkv, d, nblk = 16, 2, 16, 40
+    bt = np.array([[7, -1, -1], [3, 30, 12], [0, 21, -1]], np.int32)
+    cache = PagedCache(nblk, Hkv, B, d, fill=0xABCD)
+    T = int(q_lens.sum())
+    k, v = _bits(rng, (T, Hkv, d)), _bits(rng, (T, Hkv, d))
+    append_kv(cache, bt, q_lens, ctx_lens, k, v)
+    seq, pos = token_positions(q_lens, ctx_lens)
+    written = set()
+    for t in range(T):
+        blk, slot = bt[seq[t], pos[t] // B], pos[t] % B
+        assert np.array_equal(cache.block(blk)[0, :, slot], k[t])
+        assert np.array_equal(cache.block(blk)[1, :, slot], v[t])
+        written.add((blk, slot))
+    for blk in range(nblk):
+        for slot in range(B):
+            if (blk, slot) not in written:
+                assert (cache.block(blk)[:, :, slot] == 0xABCD).all()
+
+
+def test_uniform_keys_give_mean_of_admitted_values():
+    rng = np.random.default_rng(2)
+    L, d = 50, 32
+    K = np.tile(rng.standard_normal((1, d)), (L, 1))
+    V = rng.standard_normal((L, d))
+    pos = np.array([0, 7, 49, 30])
+    q = rng.standard_normal((4, d))
+    for window in (0, 8):
+        o = attend_contiguous(q, pos, K, V, 0.125, window)
+        for i, p in enumerate(pos):
+            lo = max(0, p - window + 1) if window else 0
+            assert np.allclose(o[i], V[lo:p + 1].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_single_admitted_key_returns_its_value():
+    rng = np.random.default_rng(3)
+    K, V = rng.standard_normal((20, 16)), rng.standard_normal((20, 16))
+    q = rng.standard_normal((3, 16))
+    o = attend_contiguous(q[:1], [0], K, V, 1.0)                  # position 0
+    assert np.array_equal(o[0], V[0])
+    o = attend_contiguous(q, [4, 11, 19], K, V, 1.0, window=1)    # window of one
+    assert np.array_equal(o, V[[4, 11, 19]])
+
+
+def _run(w, cache=None, write_ctx=True):
+    cache = cache or PagedCache(w.n_blocks, w.n_kv_heads, w.block_size, w.head_dim)
+    if write_ctx:
+        for s, kc, vc in w.contexts():
+            cache.write_positions(w.block_tables[s], np.arange(kc.shape[0]), kc, vc)
+    q, k, v = w.qkv()
+    _, _, o = splitfuse_pass(cache, w.block_tables, w.q_lens, w.ctx_lens, q, k, v,
+                             w.rope_theta, w.softmax_scale, w.sliding_window)
+    return cache, o
+
+
+def test_block_permutation_leaves_output_bit_identical():
+    w = W.config1()
+    _, o1 = _run(w)
+    _, o2 = _run(w.with_permuted_blocks(99))
+    assert not np.array_equal(w.block_tables, w.with_permuted_blocks(99).block_tables)
+    assert np.array_equal(o1, o2)
+
+
+def test_chunked_prefill_equals_one_shot():
+    one = W.prompt_chunks(4, 2, 64, 16, 200, 200, seed=21)
+    many = W.prompt_chunks(4, 2, 64, 16, 200, 48, seed=21)
+    c1, o1 = _run(one[0], write_ctx=False)
+    c2 = None
+    outs = []
+    for w in many:
+        c2, o = _run(w, c2, write_ctx=False)
+        outs.append(o)
+    o2 = np.concatenate(outs)
+    assert set(c1.blocks) == set(c2.blocks)
+    for b in c1.blocks:
+        assert np.array_equal(c1.blocks[b], c2.blocks[b])
+    assert np.abs(o1 - o2).max() <= 1e-12
+
+
+def test_window_at_least_length_equals_no_window():
+    w = W.config1()
+    _, o0 = _run(w)
+    w2 = W.config1()
+    w2.sliding_window = 64
+    _, o1 = _run(w2)
+    assert np.array_equal(o0, o1)
+
+
+def test_gqa_equals_mha_with_replicated_kv():
+    rng = np.random.default_rng(5)
+    Hq, Hkv, d, B = 4, 2, 16, 16
+    q_lens, ctx_lens = np.array([6, 1]), np.array([3, 20])
+    bt = np.array([[0, -1], [1, 2]], np.int32)
+    T = 7
+    k, v = _bits(rng, (T, Hkv, d)), _bits(rng, (T, Hkv, d))
+    Q = _bits(rng, (T, Hq, d))
+    kc, vc = _bits(rng, (20, Hkv, d)), _bits(rng, (20, Hkv, d))
+    g = PagedCache(4, Hkv, B, d)
+    m = PagedCache(4, Hq, B, d)
+    g.write_positions(bt[0], np.arange(3), kc[:3], vc[:3])
+    g.write_positions(bt[1], np.arange(20), kc, vc)
+    m.write_positions(bt[0], np.arange(3), np.repeat(kc[:3], 2, 1), np.repeat(vc[:3], 2, 1))
+    m.write_positions(bt[1], np.arange(20), np.repeat(kc, 2, 1), np.repeat(vc, 2, 1))
+    append_kv(g, bt, q_lens, ctx_lens, k, v)
+    append_kv(m, bt, q_lens, ctx_lens, np.repeat(k, 2, 1), np.repeat(v, 2, 1))
+    og = ragged_attention(g, bt, q_lens, ctx_lens, Q, 0.25)
+    om = ragged_attention(m, bt, q_lens, ctx_lens, Q, 0.25)
+    assert np.array_equal(og, om)
+
+
+def test_sampled_rows_equal_full_rows():
+    w = W.config1()
+    c, o = _run(w)
+    c2, _ = _run(w, write_ctx=True)
+    q, _, _ = w.qkv()
+    from oracle import rotate_half
+    _, pos = token_positions(w.q_lens, w.ctx_lens)
+    qr = rotate_half(q, pos, w.rope_theta)
+    tok = np.array([0, 39, 40, 41, 63])
+    s = ragged_attention(c, w.block_tables, w.q_lens, w.ctx_lens, qr, w.softmax_scale, 0, tok)
+    assert np.abs(s[tok] - o[tok]).max() <= 1e-12
+    assert np.isnan(s[1]).all()
