@@ -1,0 +1,386 @@
+"""Benchmark of the ragged paged-KV attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fg|reference] [--config 2]
+
+One step = one Dynamic SplitFuse forward pass of the attention path over the
+Llama-2-7B-shape SplitFuse snapshot (32/32 heads, d=128, block 64, budget
+2048 = 31 decodes + one 2017-token prompt chunk): batch put (metadata upload),
+rotary + paged append, ragged attention (+ split-KV combine). Inputs are
+resident in HBM when timing starts; L2 is flushed (256 MB write) between
+steps, outside the timed events. Prints one JSON line (rank 0).
+
+With N > 1 (torchrun) every rank runs its own replica of the step on its own
+GPU (the path has no exchange step, so no collective is on the data path);
+value = all ranks' tokens / the slowest rank's time.
+
+--impl reference times the float64 oracle on the host cores instead, on a
+bounded sample of the same workload per step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ragged-attention tokens/s at Llama-2-7B shape; % of HBM/tensor roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+def world():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(backend: str):
+    import datetime
+    import torch.distributed as dist
+    rank, ws, _ = world()
+    if ws > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, rank=rank, world_size=ws,
+                                timeout=datetime.timedelta(seconds=120))
+    return rank, ws
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# roofline accounting (algorithmic bytes and flops of one pass)
+# ---------------------------------------------------------------------------
+def algorithmic_work(w):
+    """Bytes each step must move at minimum and attention flops.
+
+    attention bytes: every admitted cached K and V row read once per kv head
+    (GQA sharing counted once), Q read and O written once;
+    append bytes: new K, V read and written to the cache, Q read, Q_rot written.
+    flops: 4 * d * Hq per admitted (query, key) pair (QK^T and PV)."""
+    Hq, Hkv, d, W = w.n_q_heads, w.n_kv_heads, w.head_dim, w.sliding_window
+    kv_rows = 0
+    pairs = 0
+    for q, c in zip(w.q_lens.tolist(), w.ctx_lens.tolist()):
+        p = np.arange(c, c + q, dtype=np.int64)
+        lo = np.maximum(0, p - W + 1) if W > 0 else np.zeros_like(p)
+        kv_rows += int(p[-1] + 1 - lo[0])
+        pairs += int((p - lo + 1).sum())
+    T = w.n_tokens
+    attn_bytes = kv_rows * Hkv * d * 2 * 2 + T * Hq * d * 2 * 2
+    append_bytes = T * Hkv * d * 2 * 2 * 2 + T * Hq * d * 2 * 2
+    flops = 4 * d * Hq * pairs
+    return {"attn_bytes": attn_bytes, "append_bytes": append_bytes, "flops": flops,
+            "pairs": pairs, "kv_rows": kv_rows}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return j["hbm_gbs"], j["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True,
+                                     text=True, timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[2 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_sample(w, max_chunk_rows=192):
+    """A bounded slice of the workload for the float64 oracle: every decode
+    sequence plus the first ``max_chunk_rows`` tokens of each prompt chunk
+    (each such slice is itself a valid, shorter chunk at the same context)."""
+    from ragged_paged_kv_b200 import workloads as W
+    q = np.minimum(w.q_lens, max_chunk_rows)
+    sub = W.Workload(name=w.name + "_sample", n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                     head_dim=w.head_dim, block_size=w.block_size, n_blocks=w.n_blocks,
+                     rope_theta=w.rope_theta, sliding_window=w.sliding_window, seq_ids=w.seq_ids,
+                     q_lens=q.astype(np.int32), ctx_lens=w.ctx_lens, block_tables=w.block_tables,
+                     seed=w.seed, budget=int(q.sum()))
+    return sub
+
+
+def time_oracle(w, reps=1):
+    """Seconds per oracle pass (rotary + append + attention) over workload w,
+    with the prior context written into a fresh oracle cache first (untimed)."""
+    from oracle import PagedCache
+    from oracle.forward import splitfuse_pass
+    q, k, v = w.qkv()
+    times = []
+    for _ in range(reps):
+        pc = PagedCache(w.n_blocks, w.n_kv_heads, w.block_size, w.head_dim, fill=0)
+        for s, kc, vc in w.contexts():
+            pc.write_positions(w.block_tables[s], np.arange(kc.shape[0]), kc, vc)
+        t0 = time.perf_counter()
+        splitfuse_pass(pc, w.block_tables, w.q_lens, w.ctx_lens, q, k, v, w.rope_theta,
+                       w.softmax_scale, w.sliding_window)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(w):
+    sub = oracle_sample(w, max_chunk_rows=768)
+    t = time_oracle(sub, reps=1)[0]
+    return {"value": sub.n_tokens / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{sub.n_tokens} tokens: all {int((w.q_lens == 1).sum())} decodes + first "
+                      f"{int(sub.q_lens.max())} tokens of each prompt chunk, float64 numpy, "
+                      f"{t:.2f} s"}
+
+
+def run_reference(args, w, rank, ws):
+    if rank != 0:
+        return 0
+    sub = oracle_sample(w)
+    for _ in range(args.warmup):
+        time_oracle(sub)
+    times = [time_oracle(sub)[0] for _ in range(args.steps)]
+    ms = 1000 * sum(times) / len(times)
+    value = sub.n_tokens / (ms / 1000)
+    cores = blas_threads()
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "tokens": w.n_tokens, "seqs": w.n_seqs,
+                       "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                       "block_size": w.block_size, "note": w.note},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{sub.n_tokens} tokens per step (all decodes + first "
+                                       f"{int(sub.q_lens.max())} tokens of each chunk)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def run_fg(args, w, rank, ws, local_rank):
+    import torch
+    from ragged_paged_kv_b200 import fg, fixtures
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim, device=dev)
+    fixtures.fill(cache.tensor, 0)
+    fixtures.write_context(w, cache.tensor)
+    batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+    q, k, v = fixtures.qkv_device(w, dev)
+    q_rot, out = torch.empty_like(q), torch.empty_like(q)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    def step(ev):
+        ev[0].record(stream)
+        batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, stream)
+        fg.rotary_kv_append(cache, batch, q, k, v, q_rot, w.n_q_heads, w.rope_theta, stream)
+        ev[1].record(stream)
+        fg.ragged_attention(cache, batch, q_rot, out, w.n_q_heads, w.softmax_scale,
+                            w.sliding_window, stream)
+        ev[2].record(stream)
+
+    def flush_l2():
+        with torch.cuda.stream(stream):
+            flush.zero_()
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for _ in range(args.warmup):
+        step(mk())
+        flush_l2()
+    torch.cuda.synchronize()
+    batch.device_status(stream)
+
+    evs = [mk() for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        for i in range(args.steps):
+            step(evs[i])
+            flush_l2()
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    ms_local = sum(step_ms) / len(step_ms)
+    ms = max_over_ranks(ms_local, dev)
+    attn_ms_mean = max_over_ranks(sum(attn_ms) / len(attn_ms), dev)
+    batch.device_status(stream)
+    info = batch.plan_info()
+
+    # end to end through the public API from pinned host buffers
+    host_in = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v))}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dev_bufs = {"q": q, "k": k, "v": v, "q_rot": q_rot, "out": out}
+
+    def e2e_step():
+        batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, stream)
+        fg.forward_host(cache, batch, host_in, dev_bufs, host_out, w.n_q_heads, w.rope_theta,
+                        w.softmax_scale, w.sliding_window, stream)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+        flush_l2()
+    torch.cuda.synchronize()
+    e2e_ev = [mk() for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        e2e_ev[i][0].record(stream)
+        e2e_step()
+        e2e_ev[i][1].record(stream)
+        flush_l2()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / args.steps, dev)
+    meta_bytes = 4 * (3 * w.n_seqs + 2 + w.n_tokens +
+                      sum(w.blocks_used(s) for s in range(w.n_seqs)))
+    h2d = sum(t.numel() * 2 for t in host_in.values()) + meta_bytes
+    d2h = host_out.numel() * 2
+
+    if rank != 0:
+        return 0
+    work = algorithmic_work(w)
+    hbm, tf, src = load_peaks()
+    achieved = work["attn_bytes"] / (attn_ms_mean / 1000) / 1e9
+    tokens = w.n_tokens * ws
+    line = {
+        "metric": METRIC, "value": tokens / (ms / 1000), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name} (Llama-2-7B attention shape)", "tokens_per_gpu": w.n_tokens,
+                   "seqs": w.n_seqs, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+                   "head_dim": w.head_dim, "block_size": w.block_size, "pool_blocks": w.n_blocks,
+                   "note": w.note, "l2": "flushed between steps (256 MB write, outside the events)",
+                   "parallelism": f"replicas x{ws}"},
+        "roofline": {"kernel": "ragged attention (work units + split-KV combine)", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "peak_source": src,
+                     "attn_ms": attn_ms_mean, "algorithmic_bytes": work["attn_bytes"],
+                     "flops": work["flops"],
+                     "tflops_achieved": work["flops"] / (attn_ms_mean / 1000) / 1e12,
+                     "step_roofline_ms": 1000 * max((work["attn_bytes"] + work["append_bytes"]) / (hbm * 1e9),
+                                                    work["flops"] / (tf * 1e12))},
+        "e2e": {"value": tokens / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * (1 + info["launches"]),
+        "plan": info,
+        "clocks": clocks.summary(),
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["fg", "reference"], default="fg")
+    ap.add_argument("--config", type=int, default=2, help="workload number (2 = the headline)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--compact-pool", action="store_true",
+                    help="size the block pool to what the batch uses (small ncu captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from ragged_paged_kv_b200 import workloads as W
+    w = W.CONFIGS[args.config]()
+    if args.compact_pool:
+        need = sum(w.blocks_used(s) for s in range(w.n_seqs))
+        w = W._make(w.name, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.seq_ids,
+                    w.q_lens, w.ctx_lens, w.seed, w.budget, n_blocks=need + 16,
+                    window=w.sliding_window, note=w.note + "; compact pool")
+    if args.impl == "reference":
+        rank, ws = init_dist("gloo")
+        rc = run_reference(args, w, rank, ws)
+    else:
+        import torch
+        rank, ws = init_dist("nccl")
+        rc = run_fg(args, w, rank, ws, world()[2])
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,195 @@
+/*
+ * fg.h - C ABI of the B200 ragged paged-KV attention library (libfg).
+ *
+ * One Dynamic SplitFuse forward pass of attention: a ragged batch of prompt
+ * chunks and single-token decodes, at most a fixed token budget ("DeepSpeed-
+ * FastGen — paper by Holmes et al. (2024)", Summary: every forward pass is
+ * kept at a fixed token count; long prompts are cut into chunks spread over
+ * several iterations; short prompts and generation tokens fill the rest). For
+ * that batch the library
+ *   1. rotates Q and K with rotary position embedding,
+ *   2. appends the new K and V into a blocked (paged) KV cache through
+ *      per-sequence block tables (same page, Key points: the KV cache is
+ *      blocked as in PagedAttention),
+ *   3. runs one ragged causal attention of every new token over its
+ *      sequence's cached context.
+ *
+ * Conventions shared by every call
+ *   - Types: all tensors are bf16 (16-bit words), row-major, densely packed.
+ *     T = tokens in the batch, Hq / Hkv = query / key-value heads,
+ *     d = head_dim, B = block_size.
+ *   - Pointers marked "device" must point to memory of the current CUDA
+ *     device; "host" pointers are ordinary CPU memory that the call only
+ *     reads during the call (nothing is retained).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Device work is asynchronous on it; calls that touch the same
+ *     cache / batch must be issued on one stream, in the order
+ *     put -> rotary_kv_append -> ragged_attention.
+ *   - Every call returns an fg_status and never aborts the process. On
+ *     failure nothing was launched and no output was written;
+ *     fg_last_error() gives a thread-local, human-readable reason.
+ *   - Handles are owned by the caller and released by the matching
+ *     *_destroy. A handle may be used by one host thread at a time.
+ */
+#ifndef FG_H_
+#define FG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fg_status {
+  FG_OK = 0,
+  FG_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad handle          */
+  FG_ERR_OUT_OF_RANGE = 2,  /* a block id outside [0, n_blocks)                 */
+  FG_ERR_ALIAS = 3,         /* two writes to one cache slot, duplicate seq ids  */
+  FG_ERR_CAPACITY = 4,      /* batch larger than the handle was created for     */
+  FG_ERR_UNSUPPORTED = 5,   /* head_dim / block_size / head ratio not built     */
+  FG_ERR_CUDA = 6,          /* a CUDA runtime call failed (no device, OOM ...)  */
+  FG_ERR_DEVICE_CHECK = 7,  /* a kernel found an out-of-range index and skipped */
+  FG_ERR_TIMEOUT = 8        /* a bounded device wait gave up                    */
+} fg_status;
+
+typedef struct fg_kv_cache fg_kv_cache;         /* opaque */
+typedef struct fg_ragged_batch fg_ragged_batch; /* opaque */
+
+/* ------------------------------------------------------------------------ */
+/* Paged KV cache (Key points: blocked KV cache as in PagedAttention)        */
+/* ------------------------------------------------------------------------ */
+
+/* Allocate a cache of n_blocks blocks on the current device with cudaMalloc.
+ * Layout (bf16 words): [n_blocks][2 (0 = K, 1 = V)][n_kv_heads][block_size]
+ * [head_dim]; one (block, K|V, head) tile is block_size*head_dim contiguous
+ * words. Contents are left uninitialised. Supported: head_dim in {64, 128},
+ * block_size in {16, 32, 64, 128}, n_kv_heads in [1, 256], n_blocks >= 1,
+ * else FG_ERR_UNSUPPORTED / FG_ERR_INVALID_ARG. Offsets are 64-bit, so a pool
+ * may fill the whole of a 180 GB device. */
+fg_status fg_kv_cache_create(int32_t block_size, int32_t n_blocks, int32_t n_kv_heads,
+                             int32_t head_dim, fg_kv_cache** out);
+
+/* Same, over caller-owned device memory (e.g. a torch tensor) of `bytes`
+ * bytes at `dev_ptr` (16-byte aligned, at least the size above). The
+ * memory is borrowed: it must outlive the handle and is never freed here. */
+fg_status fg_kv_cache_create_external(int32_t block_size, int32_t n_blocks, int32_t n_kv_heads,
+                                      int32_t head_dim, void* dev_ptr, size_t bytes,
+                                      fg_kv_cache** out);
+
+/* Base device pointer and element strides of the 5-d layout above
+ * (strides_elems[0] = block, [1] = K|V, [2] = head, [3] = slot, [4] = dim). */
+fg_status fg_kv_cache_layout(const fg_kv_cache* cache, void** base, int64_t strides_elems[5]);
+
+/* Releases the handle and (for fg_kv_cache_create) the pool. Waits for the
+ * device first. NULL is accepted. */
+fg_status fg_kv_cache_destroy(fg_kv_cache* cache);
+
+/* ------------------------------------------------------------------------ */
+/* Ragged batch (Summary: a fixed budget filled with prompt chunks and       */
+/* generation tokens)                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* A reusable holder for one batch's metadata, sized for at most max_tokens
+ * new tokens, max_seqs sequences and max_blocks_per_seq blocks per sequence.
+ * Device buffers are allocated on the first successful put. */
+fg_status fg_ragged_batch_create(int32_t max_tokens, int32_t max_seqs, int32_t max_blocks_per_seq,
+                                 fg_ragged_batch** out);
+
+/* Describe the next forward pass. Host arrays, all of length n_seqs:
+ *   seq_ids   caller's sequence ids (distinct; used only for validation),
+ *   q_lens    new tokens of each sequence (>= 1): prompt-chunk length or 1,
+ *   ctx_lens  tokens already in the cache before this pass (>= 0);
+ * block_tables: host int32 [n_seqs][block_table_stride]; row s lists the
+ * physical blocks of sequence s in logical order and must hold at least
+ * ceil((ctx_lens[s] + q_lens[s]) / block_size) valid ids; entries past that
+ * are ignored. Token rows of q/k/v/out are packed in this sequence order,
+ * sequence s's new tokens sitting at absolute positions ctx_lens[s] ..
+ * ctx_lens[s] + q_lens[s] - 1. n_seqs == 0 describes an empty pass.
+ * Checks, all before any device work: sizes within the handle's capacity
+ * (FG_ERR_CAPACITY), q_lens >= 1 and ctx_lens >= 0 (FG_ERR_INVALID_ARG),
+ * used block ids inside the cache (FG_ERR_OUT_OF_RANGE), no cache slot
+ * written twice, no block repeated within one table, no new token written
+ * into a slot that another sequence of the batch reads, distinct seq_ids
+ * (FG_ERR_ALIAS). The packed metadata is copied to the device
+ * asynchronously on `stream` from a pinned staging buffer; a later put on
+ * the same handle first waits for that copy. */
+fg_status fg_ragged_batch_put(fg_ragged_batch* batch, const fg_kv_cache* cache, int32_t n_seqs,
+                              const int32_t* seq_ids, const int32_t* q_lens,
+                              const int32_t* ctx_lens, const int32_t* block_tables,
+                              int32_t block_table_stride, void* stream);
+
+/* Tokens and sequences of the last successful put. */
+fg_status fg_ragged_batch_shape(const fg_ragged_batch* batch, int32_t* n_tokens, int32_t* n_seqs);
+
+fg_status fg_ragged_batch_destroy(fg_ragged_batch* batch);
+
+/* ------------------------------------------------------------------------ */
+/* Step 1 + 2: rotary on Q/K, append K_rot and V into the cache              */
+/* ------------------------------------------------------------------------ */
+
+/* q: device [T][n_q_heads][d], k and v: device [T][Hkv][d], q_rot: device
+ * [T][n_q_heads][d] (may equal q for in-place). For token at position p and
+ * frequency i < d/2: inv_freq_i = 1 / rope_theta^(2i/d), a = p * inv_freq_i
+ * in double; c, s = cos(a), sin(a) by the host C library in double, rounded
+ * once to float; pairs (i, i + d/2) are rotated in double,
+ *   y_i = x_i c - x_{i+d/2} s,   y_{i+d/2} = x_{i+d/2} c + x_i s,
+ * and each result is rounded once to bf16 (ties to even). The pages name the
+ * HuggingFace LLaMA / Mistral families (Key points), which use this
+ * rotate-half pairing. K_rot and V are bit-copied to slot p % B of block
+ * block_table[s][p / B]; no other cache word changes. n_q_heads must be a
+ * multiple of the cache's n_kv_heads. The first call for a (rope_theta,
+ * position range) builds or grows the cos/sin table on the host and uploads
+ * it (synchronous, allocating); later calls reuse it. */
+fg_status fg_rotary_kv_append(fg_kv_cache* cache, const fg_ragged_batch* batch, const void* q,
+                              const void* k, const void* v, void* q_rot, int32_t n_q_heads,
+                              double rope_theta, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Step 3: one ragged causal attention over every sequence's cached context  */
+/* ------------------------------------------------------------------------ */
+
+/* q_rot: device [T][n_q_heads][d] (rotated queries); out: device
+ * [T][n_q_heads][d]. Query head h reads kv head h / (n_q_heads / Hkv). The
+ * token at position p attends to the cached positions k with
+ * max(0, p - sliding_window + 1) <= k <= p (sliding_window = 0: no window),
+ *   out = sum_k exp(z_k - m) V_k / sum_k exp(z_k - m),
+ *   z_k = softmax_scale * <q, K_k>,  m = max_k z_k,
+ * with bf16 operands, fp32 accumulation and fp32 softmax. Must follow the
+ * fg_rotary_kv_append of the same batch on the same stream (a token sees its
+ * own K/V). Long contexts are split across thread blocks and merged by a
+ * log-sum-exp combine; the split workspace is owned by the batch handle and
+ * grown (cudaMalloc, after a device synchronize) when a pass needs more. */
+fg_status fg_ragged_attention(const fg_kv_cache* cache, fg_ragged_batch* batch, const void* q_rot,
+                              void* out, int32_t n_q_heads, float softmax_scale,
+                              int32_t sliding_window, void* stream);
+
+/* Work plan of the batch's last fg_ragged_attention call, for profiling:
+ * info[0] = general-path units, info[1] = split-KV decode units,
+ * info[2] = tensor-core units, info[3] = combine groups, info[4] = partial
+ * rows in the split workspace, info[5] = kernels launched by that call,
+ * info[6..7] = 0. */
+fg_status fg_attention_plan_info(const fg_ragged_batch* batch, int32_t info[8]);
+
+/* Reads (and clears) the batch's device error word after synchronising
+ * `stream`: FG_OK, or FG_ERR_DEVICE_CHECK if a kernel met an index outside
+ * its buffers (the access was skipped), or FG_ERR_TIMEOUT. */
+fg_status fg_device_status(fg_ragged_batch* batch, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Host-only helpers                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* The float cos/sin table rotary uses, for positions pos_begin ..
+ * pos_begin + n_pos - 1: cos_out/sin_out are host float [n_pos][head_dim/2].
+ * No device needed. */
+fg_status fg_rotary_table(double rope_theta, int32_t head_dim, int32_t pos_begin, int32_t n_pos,
+                          float* cos_out, float* sin_out);
+
+const char* fg_status_string(fg_status status);
+const char* fg_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FG_H_ */

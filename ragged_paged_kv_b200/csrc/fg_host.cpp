@@ -1,0 +1,671 @@
+// Host side of libfg: handles, argument validation, batch metadata packing,
+// the rotary cos/sin table, work planning and kernel launch sequencing.
+//
+// Everything the kernels need about a ragged batch is packed by
+// fg_ragged_batch_put into one int32 buffer and sent with a single
+// asynchronous host-to-device copy; fg_ragged_attention plans its work units
+// on the host (integer work only) and sends them the same way.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/fg.h"
+#include "fg_internal.h"
+#include "fg_plan.h"
+
+using fg::BatchView;
+using fg::CacheView;
+using fg::CombineItem;
+using fg::WorkItem;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+fg_status fail(fg_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+fg_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FG_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define FG_CUDA(call)                                   \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A pinned host staging area with two halves used in turn; before a half is
+// rewritten the host waits for the copy that last read it.
+struct Staging {
+  void* host[2] = {nullptr, nullptr};
+  size_t bytes = 0;
+  cudaEvent_t done[2] = {nullptr, nullptr};
+  bool pending[2] = {false, false};
+  int next = 0;
+
+  fg_status reserve(size_t need) {
+    if (need <= bytes) return FG_OK;
+    for (int i = 0; i < 2; ++i) {
+      if (pending[i]) FG_CUDA(cudaEventSynchronize(done[i]));
+      pending[i] = false;
+      if (host[i]) cudaFreeHost(host[i]);
+      host[i] = nullptr;
+    }
+    size_t cap = std::max<size_t>(need, 4096);
+    for (int i = 0; i < 2; ++i) {
+      FG_CUDA(cudaHostAlloc(&host[i], cap, cudaHostAllocDefault));
+      if (!done[i]) FG_CUDA(cudaEventCreateWithFlags(&done[i], cudaEventDisableTiming));
+    }
+    bytes = cap;
+    return FG_OK;
+  }
+  // Returns a half that is free to write.
+  fg_status acquire(void** out, int* idx) {
+    const int i = next;
+    if (pending[i]) FG_CUDA(cudaEventSynchronize(done[i]));
+    pending[i] = false;
+    *out = host[i];
+    *idx = i;
+    next ^= 1;
+    return FG_OK;
+  }
+  fg_status copy(int i, void* dst, size_t n, cudaStream_t st) {
+    if (n) FG_CUDA(cudaMemcpyAsync(dst, host[i], n, cudaMemcpyHostToDevice, st));
+    FG_CUDA(cudaEventRecord(done[i], st));
+    pending[i] = true;
+    return FG_OK;
+  }
+  void release() {
+    for (int i = 0; i < 2; ++i) {
+      if (pending[i]) cudaEventSynchronize(done[i]);
+      if (host[i]) cudaFreeHost(host[i]);
+      if (done[i]) cudaEventDestroy(done[i]);
+      host[i] = nullptr;
+      done[i] = nullptr;
+    }
+  }
+};
+
+}  // namespace
+
+struct fg_kv_cache {
+  int32_t block_size = 0, n_blocks = 0, n_kv_heads = 0, head_dim = 0;
+  void* base = nullptr;
+  size_t bytes = 0;
+  bool owned = false;
+  int device = 0;
+  // rotary table [rope_npos][head_dim / 2] of (cos, sin)
+  double rope_theta = 0.0;
+  int32_t rope_npos = 0;
+  float2* rope = nullptr;
+};
+
+struct fg_ragged_batch {
+  int32_t max_tokens = 0, max_seqs = 0, max_blocks_per_seq = 0;
+  int device = -1;
+  // device metadata + error word
+  int32_t* dmeta = nullptr;
+  size_t dmeta_words = 0;
+  int32_t* derr = nullptr;
+  Staging meta_stage;
+  // last put
+  const fg_kv_cache* cache = nullptr;
+  uint64_t put_gen = 0;
+  int32_t n_seqs = 0, n_tokens = 0, max_pos = -1;
+  std::vector<int32_t> q_lens, ctx_lens;
+  BatchView view{};
+  // alias-check scratch, indexed by block id
+  std::vector<uint64_t> stamp;
+  std::vector<int32_t> head;
+  // attention plan
+  fg::Plan plan;
+  uint64_t plan_key[4] = {~0ull, 0, 0, 0};
+  void* dplan = nullptr;
+  size_t dplan_bytes = 0;
+  Staging plan_stage;
+  int32_t last_launches = 0;
+  // split-KV partials
+  float* ws = nullptr;
+  size_t ws_bytes = 0;
+};
+
+// ---------------------------------------------------------------------------
+// rotary table
+// ---------------------------------------------------------------------------
+static void build_rope_rows(double theta, int d, int p0, int n, float* c, float* s, int ld) {
+  const int half = d / 2;
+  std::vector<double> inv(half);
+  for (int i = 0; i < half; ++i) inv[i] = 1.0 / std::pow(theta, (2.0 * i) / (double)d);
+  for (int r = 0; r < n; ++r) {
+    const double p = (double)(p0 + r);
+    for (int i = 0; i < half; ++i) {
+      const double a = p * inv[i];
+      c[(size_t)r * ld + i] = (float)std::cos(a);
+      s[(size_t)r * ld + i] = (float)std::sin(a);
+    }
+  }
+}
+
+extern "C" fg_status fg_rotary_table(double rope_theta, int32_t head_dim, int32_t pos_begin,
+                                     int32_t n_pos, float* cos_out, float* sin_out) {
+  if (!(rope_theta > 0.0) || head_dim <= 0 || (head_dim & 1) || pos_begin < 0 || n_pos < 0 ||
+      (n_pos > 0 && (!cos_out || !sin_out)))
+    return fail(FG_ERR_INVALID_ARG, "fg_rotary_table: bad argument");
+  build_rope_rows(rope_theta, head_dim, pos_begin, n_pos, cos_out, sin_out, head_dim / 2);
+  return FG_OK;
+}
+
+static fg_status ensure_rope(fg_kv_cache* c, double theta, int32_t max_pos) {
+  if (c->rope && c->rope_theta == theta && max_pos < c->rope_npos) return FG_OK;
+  int64_t need = (int64_t)max_pos + 1;
+  int64_t cap = 4096;
+  while (cap < need) cap *= 2;
+  const int half = c->head_dim / 2;
+  std::vector<float> cs((size_t)cap * half), sn((size_t)cap * half);
+  build_rope_rows(theta, c->head_dim, 0, (int)cap, cs.data(), sn.data(), half);
+  std::vector<float2> tab((size_t)cap * half);
+  for (size_t i = 0; i < tab.size(); ++i) tab[i] = make_float2(cs[i], sn[i]);
+  float2* dnew = nullptr;
+  FG_CUDA(cudaMalloc(&dnew, tab.size() * sizeof(float2)));
+  cudaError_t e = cudaMemcpy(dnew, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(dnew);
+    return cuda_fail(e, "rotary table upload");
+  }
+  if (c->rope) {
+    FG_CUDA(cudaDeviceSynchronize());  // earlier launches may still read the old table
+    cudaFree(c->rope);
+  }
+  c->rope = dnew;
+  c->rope_npos = (int32_t)cap;
+  c->rope_theta = theta;
+  return FG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// cache
+// ---------------------------------------------------------------------------
+static fg_status check_cache_shape(int32_t B, int32_t nb, int32_t hkv, int32_t d) {
+  if (nb < 1 || hkv < 1) return fail(FG_ERR_INVALID_ARG, "n_blocks and n_kv_heads must be >= 1");
+  if (hkv > 256) return fail(FG_ERR_UNSUPPORTED, "n_kv_heads %d > 256", hkv);
+  if (d != 64 && d != 128) return fail(FG_ERR_UNSUPPORTED, "head_dim %d not in {64, 128}", d);
+  if (B != 16 && B != 32 && B != 64 && B != 128)
+    return fail(FG_ERR_UNSUPPORTED, "block_size %d not in {16, 32, 64, 128}", B);
+  return FG_OK;
+}
+
+static size_t cache_bytes(int32_t B, int32_t nb, int32_t hkv, int32_t d) {
+  return (size_t)nb * 2 * (size_t)hkv * (size_t)B * (size_t)d * 2;
+}
+
+extern "C" fg_status fg_kv_cache_create(int32_t block_size, int32_t n_blocks, int32_t n_kv_heads,
+                                        int32_t head_dim, fg_kv_cache** out) {
+  if (!out) return fail(FG_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  fg_status st = check_cache_shape(block_size, n_blocks, n_kv_heads, head_dim);
+  if (st) return st;
+  auto* c = new fg_kv_cache;
+  c->block_size = block_size;
+  c->n_blocks = n_blocks;
+  c->n_kv_heads = n_kv_heads;
+  c->head_dim = head_dim;
+  c->bytes = cache_bytes(block_size, n_blocks, n_kv_heads, head_dim);
+  c->owned = true;
+  cudaError_t e = cudaGetDevice(&c->device);
+  if (e == cudaSuccess) e = cudaMalloc(&c->base, c->bytes);
+  if (e != cudaSuccess) {
+    delete c;
+    return cuda_fail(e, "fg_kv_cache_create: cudaMalloc of the block pool");
+  }
+  *out = c;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_kv_cache_create_external(int32_t block_size, int32_t n_blocks,
+                                                 int32_t n_kv_heads, int32_t head_dim,
+                                                 void* dev_ptr, size_t bytes, fg_kv_cache** out) {
+  if (!out) return fail(FG_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  fg_status st = check_cache_shape(block_size, n_blocks, n_kv_heads, head_dim);
+  if (st) return st;
+  if (!dev_ptr || !aligned16(dev_ptr))
+    return fail(FG_ERR_INVALID_ARG, "dev_ptr must be a 16-byte aligned device pointer");
+  const size_t need = cache_bytes(block_size, n_blocks, n_kv_heads, head_dim);
+  if (bytes < need)
+    return fail(FG_ERR_CAPACITY, "external cache has %zu bytes, layout needs %zu", bytes, need);
+  auto* c = new fg_kv_cache;
+  c->block_size = block_size;
+  c->n_blocks = n_blocks;
+  c->n_kv_heads = n_kv_heads;
+  c->head_dim = head_dim;
+  c->bytes = need;
+  c->base = dev_ptr;
+  c->owned = false;
+  if (cudaGetDevice(&c->device) != cudaSuccess) c->device = -1;
+  *out = c;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_kv_cache_layout(const fg_kv_cache* c, void** base, int64_t strides[5]) {
+  if (!c || !base || !strides) return fail(FG_ERR_INVALID_ARG, "NULL argument");
+  *base = c->base;
+  strides[4] = 1;
+  strides[3] = c->head_dim;
+  strides[2] = (int64_t)c->block_size * c->head_dim;
+  strides[1] = strides[2] * c->n_kv_heads;
+  strides[0] = strides[1] * 2;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_kv_cache_destroy(fg_kv_cache* c) {
+  if (!c) return FG_OK;
+  if (c->owned || c->rope) cudaDeviceSynchronize();
+  if (c->owned && c->base) cudaFree(c->base);
+  if (c->rope) cudaFree(c->rope);
+  delete c;
+  return FG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// ragged batch
+// ---------------------------------------------------------------------------
+extern "C" fg_status fg_ragged_batch_create(int32_t max_tokens, int32_t max_seqs,
+                                            int32_t max_blocks_per_seq, fg_ragged_batch** out) {
+  if (!out) return fail(FG_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (max_tokens < 1 || max_seqs < 1 || max_blocks_per_seq < 1)
+    return fail(FG_ERR_INVALID_ARG, "capacities must be >= 1");
+  if ((int64_t)max_seqs * max_blocks_per_seq > (int64_t)1 << 30)
+    return fail(FG_ERR_CAPACITY, "max_seqs * max_blocks_per_seq too large");
+  auto* b = new fg_ragged_batch;
+  b->max_tokens = max_tokens;
+  b->max_seqs = max_seqs;
+  b->max_blocks_per_seq = max_blocks_per_seq;
+  *out = b;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_ragged_batch_destroy(fg_ragged_batch* b) {
+  if (!b) return FG_OK;
+  if (b->dmeta || b->dplan || b->ws) cudaDeviceSynchronize();
+  b->meta_stage.release();
+  b->plan_stage.release();
+  if (b->dmeta) cudaFree(b->dmeta);
+  if (b->derr) cudaFree(b->derr);
+  if (b->dplan) cudaFree(b->dplan);
+  if (b->ws) cudaFree(b->ws);
+  delete b;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_ragged_batch_shape(const fg_ragged_batch* b, int32_t* n_tokens,
+                                           int32_t* n_seqs) {
+  if (!b) return fail(FG_ERR_INVALID_ARG, "batch is NULL");
+  if (n_tokens) *n_tokens = b->n_tokens;
+  if (n_seqs) *n_seqs = b->n_seqs;
+  return FG_OK;
+}
+
+namespace {
+
+// Every check of fg_ragged_batch_put that needs no device.
+fg_status validate_batch(fg_ragged_batch* b, const fg_kv_cache* c, int32_t S, const int32_t* ids,
+                         const int32_t* ql, const int32_t* cl, const int32_t* bt, int32_t stride,
+                         int64_t* T_out, int64_t* nblk_out, int32_t* maxpos_out) {
+  if (S < 0) return fail(FG_ERR_INVALID_ARG, "n_seqs %d < 0", S);
+  if (S > b->max_seqs) return fail(FG_ERR_CAPACITY, "n_seqs %d > max_seqs %d", S, b->max_seqs);
+  if (S > 0 && (!ids || !ql || !cl || !bt))
+    return fail(FG_ERR_INVALID_ARG, "NULL host array");
+  if (S > 0 && stride < 1) return fail(FG_ERR_INVALID_ARG, "block_table_stride %d < 1", stride);
+  const int64_t B = c->block_size;
+  int64_t T = 0, nblk = 0;
+  int32_t maxpos = -1;
+  for (int32_t s = 0; s < S; ++s) {
+    if (ql[s] < 1) return fail(FG_ERR_INVALID_ARG, "q_lens[%d] = %d < 1", s, ql[s]);
+    if (cl[s] < 0) return fail(FG_ERR_INVALID_ARG, "ctx_lens[%d] = %d < 0", s, cl[s]);
+    const int64_t L = (int64_t)cl[s] + ql[s];
+    if (L > (int64_t)1 << 30) return fail(FG_ERR_CAPACITY, "sequence %d length %lld too long", s, (long long)L);
+    const int64_t nb = (L + B - 1) / B;
+    if (nb > b->max_blocks_per_seq)
+      return fail(FG_ERR_CAPACITY, "sequence %d needs %lld blocks > max_blocks_per_seq %d", s,
+                  (long long)nb, b->max_blocks_per_seq);
+    if (nb > stride)
+      return fail(FG_ERR_INVALID_ARG, "sequence %d needs %lld blocks > block_table_stride %d", s,
+                  (long long)nb, stride);
+    T += ql[s];
+    nblk += nb;
+    maxpos = std::max<int32_t>(maxpos, (int32_t)(L - 1));
+  }
+  if (T > b->max_tokens)
+    return fail(FG_ERR_CAPACITY, "%lld tokens > max_tokens %d", (long long)T, b->max_tokens);
+  // distinct sequence ids
+  {
+    std::vector<int32_t> sid(ids, ids + S);
+    std::sort(sid.begin(), sid.end());
+    for (int32_t i = 1; i < S; ++i)
+      if (sid[i] == sid[i - 1]) return fail(FG_ERR_ALIAS, "duplicate seq_id %d", sid[i]);
+  }
+  // block ids in range; per block, the sequences that use it must not collide:
+  // a sequence writing slots [w, used) of a block conflicts with any other
+  // sequence touching slots below `used` at or above w.
+  struct Use { int32_t seq, used, wlo, next; };
+  std::vector<Use> uses;
+  uses.reserve((size_t)nblk);
+  if (b->stamp.size() != (size_t)c->n_blocks) {
+    b->stamp.assign((size_t)c->n_blocks, 0);
+    b->head.assign((size_t)c->n_blocks, -1);
+  }
+  const uint64_t gen = ++b->put_gen;
+  for (int32_t s = 0; s < S; ++s) {
+    const int64_t L = (int64_t)cl[s] + ql[s];
+    const int64_t nb = (L + B - 1) / B;
+    for (int64_t i = 0; i < nb; ++i) {
+      const int32_t blk = bt[(int64_t)s * stride + i];
+      if (blk < 0 || blk >= c->n_blocks)
+        return fail(FG_ERR_OUT_OF_RANGE, "block_tables[%d][%lld] = %d outside [0, %d)", s,
+                    (long long)i, blk, c->n_blocks);
+      const int32_t used = (int32_t)std::min<int64_t>(B, L - i * B);
+      const int64_t w0 = std::max<int64_t>(cl[s], i * B) - i * B;  // first written slot
+      const int32_t wlo = (int32_t)std::min<int64_t>(w0, used);     // == used: no write
+      Use u{s, used, wlo, -1};
+      if (b->stamp[blk] == gen) {
+        for (int32_t e = b->head[blk]; e >= 0; e = uses[e].next) {
+          const Use& o = uses[e];
+          if (o.seq == s)
+            return fail(FG_ERR_ALIAS, "block %d appears twice in the table of sequence %d", blk, s);
+          if ((u.wlo < u.used && o.used > u.wlo) || (o.wlo < o.used && u.used > o.wlo))
+            return fail(FG_ERR_ALIAS, "block %d: sequence %d and %d collide on written slots", blk,
+                        o.seq, s);
+        }
+        u.next = b->head[blk];
+      } else {
+        b->stamp[blk] = gen;
+      }
+      b->head[blk] = (int32_t)uses.size();
+      uses.push_back(u);
+    }
+  }
+  *T_out = T;
+  *nblk_out = nblk;
+  *maxpos_out = maxpos;
+  return FG_OK;
+}
+
+}  // namespace
+
+extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* c, int32_t S,
+                                         const int32_t* ids, const int32_t* ql, const int32_t* cl,
+                                         const int32_t* bt, int32_t stride, void* stream) {
+  if (!b || !c) return fail(FG_ERR_INVALID_ARG, "NULL handle");
+  int64_t T = 0, nblk = 0;
+  int32_t maxpos = -1;
+  fg_status st = validate_batch(b, c, S, ids, ql, cl, bt, stride, &T, &nblk, &maxpos);
+  if (st) {
+    b->cache = nullptr;  // the previous batch is no longer valid either
+    return st;
+  }
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  if (!b->dmeta) {
+    b->dmeta_words = 3 * (size_t)b->max_seqs + 2 + (size_t)b->max_tokens +
+                     (size_t)b->max_seqs * b->max_blocks_per_seq;
+    FG_CUDA(cudaGetDevice(&b->device));
+    FG_CUDA(cudaMalloc(&b->dmeta, b->dmeta_words * 4));
+    FG_CUDA(cudaMalloc(&b->derr, 4));
+    FG_CUDA(cudaMemset(b->derr, 0, 4));
+    st = b->meta_stage.reserve(b->dmeta_words * 4);
+    if (st) return st;
+  }
+  // pack: cu_q[S+1] ctx[S] bt_off[S+1] tok_seq[T] bt[nblk]
+  const size_t words = 3 * (size_t)S + 2 + (size_t)T + (size_t)nblk;
+  void* hp = nullptr;
+  int slot = 0;
+  st = b->meta_stage.acquire(&hp, &slot);
+  if (st) return st;
+  int32_t* h = static_cast<int32_t*>(hp);
+  int32_t* cu = h;
+  int32_t* cx = cu + S + 1;
+  int32_t* bo = cx + S;
+  int32_t* ts = bo + S + 1;
+  int32_t* bb = ts + T;
+  cu[0] = 0;
+  bo[0] = 0;
+  const int64_t B = c->block_size;
+  for (int32_t s = 0; s < S; ++s) {
+    cu[s + 1] = cu[s] + ql[s];
+    cx[s] = cl[s];
+    const int64_t nb = ((int64_t)cl[s] + ql[s] + B - 1) / B;
+    bo[s + 1] = bo[s] + (int32_t)nb;
+    std::memcpy(bb + bo[s], bt + (int64_t)s * stride, (size_t)nb * 4);
+    for (int32_t j = 0; j < ql[s]; ++j) ts[cu[s] + j] = s;
+  }
+  st = b->meta_stage.copy(slot, b->dmeta, words * 4, strm);
+  if (st) return st;
+  int32_t* d = b->dmeta;
+  b->view.cu_q = d;
+  b->view.ctx = d + S + 1;
+  b->view.bt_off = d + 2 * S + 1;
+  b->view.tok_seq = d + 3 * S + 2;
+  b->view.bt = d + 3 * S + 2 + T;
+  b->view.n_seqs = S;
+  b->view.n_tokens = (int32_t)T;
+  b->view.err = b->derr;
+  b->q_lens.assign(ql, ql + S);
+  b->ctx_lens.assign(cl, cl + S);
+  b->n_seqs = S;
+  b->n_tokens = (int32_t)T;
+  b->max_pos = maxpos;
+  b->cache = c;
+  return FG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// forward steps
+// ---------------------------------------------------------------------------
+static CacheView cache_view(const fg_kv_cache* c) {
+  CacheView v;
+  v.base = static_cast<__nv_bfloat16*>(c->base);
+  v.n_blocks = c->n_blocks;
+  v.n_kv_heads = c->n_kv_heads;
+  v.block_size = c->block_size;
+  v.head_dim = c->head_dim;
+  return v;
+}
+
+static fg_status check_pass(const fg_kv_cache* c, const fg_ragged_batch* b, int32_t hq) {
+  if (!c || !b) return fail(FG_ERR_INVALID_ARG, "NULL handle");
+  if (b->cache != c)
+    return fail(FG_ERR_INVALID_ARG, "batch was not put against this cache (or its last put failed)");
+  if (hq < 1 || hq % c->n_kv_heads)
+    return fail(FG_ERR_UNSUPPORTED, "n_q_heads %d is not a multiple of n_kv_heads %d", hq,
+                c->n_kv_heads);
+  int dev = -1;
+  if (cudaGetDevice(&dev) == cudaSuccess && b->device >= 0 && dev != b->device)
+    return fail(FG_ERR_INVALID_ARG, "current device %d is not the batch's device %d", dev, b->device);
+  return FG_OK;
+}
+
+extern "C" fg_status fg_rotary_kv_append(fg_kv_cache* c, const fg_ragged_batch* b, const void* q,
+                                         const void* k, const void* v, void* q_rot,
+                                         int32_t n_q_heads, double rope_theta, void* stream) {
+  fg_status st = check_pass(c, b, n_q_heads);
+  if (st) return st;
+  if (!(rope_theta > 0.0)) return fail(FG_ERR_INVALID_ARG, "rope_theta must be > 0");
+  if (b->n_tokens == 0) return FG_OK;
+  if (!q || !k || !v || !q_rot) return fail(FG_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_rot))
+    return fail(FG_ERR_INVALID_ARG, "q, k, v and q_rot must be 16-byte aligned");
+  st = ensure_rope(c, rope_theta, b->max_pos);
+  if (st) return st;
+  cudaError_t e = fg::launch_rotary_append(
+      cache_view(c), b->view, static_cast<const __nv_bfloat16*>(q),
+      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+      static_cast<__nv_bfloat16*>(q_rot), c->rope, n_q_heads, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rotary_append launch");
+  return FG_OK;
+}
+
+namespace {
+
+// Upload the plan for (g, window) unless the batch's current plan already is.
+fg_status prepare_plan(fg_ragged_batch* b, const fg_kv_cache* c, int32_t g, int32_t window,
+                       cudaStream_t strm) {
+  const uint64_t key[4] = {b->put_gen, (uint64_t)g, (uint64_t)(uint32_t)window,
+                           (uint64_t)c->head_dim};
+  if (std::equal(key, key + 4, b->plan_key) && b->dplan) return FG_OK;
+  fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, &b->plan);
+  const size_t bytes = b->plan.bytes();
+  if (bytes > b->dplan_bytes) {
+    if (b->dplan) FG_CUDA(cudaFreeAsync(b->dplan, strm));
+    b->dplan = nullptr;
+    const size_t cap = std::max<size_t>(bytes + bytes / 2, 1 << 16);
+    FG_CUDA(cudaMallocAsync(&b->dplan, cap, strm));
+    b->dplan_bytes = cap;
+  }
+  fg_status st = b->plan_stage.reserve(b->dplan_bytes);
+  if (st) return st;
+  void* hp = nullptr;
+  int slot = 0;
+  st = b->plan_stage.acquire(&hp, &slot);
+  if (st) return st;
+  b->plan.pack(hp);
+  st = b->plan_stage.copy(slot, b->dplan, bytes, strm);
+  if (st) return st;
+  std::copy(key, key + 4, b->plan_key);
+  return FG_OK;
+}
+
+fg_status ensure_workspace(fg_ragged_batch* b, size_t floats, cudaStream_t strm) {
+  const size_t bytes = floats * 4;
+  if (bytes <= b->ws_bytes) return FG_OK;
+  if (b->ws) FG_CUDA(cudaFreeAsync(b->ws, strm));
+  b->ws = nullptr;
+  const size_t cap = std::max<size_t>(bytes + bytes / 4, 1 << 20);
+  FG_CUDA(cudaMallocAsync(&b->ws, cap, strm));
+  b->ws_bytes = cap;
+  return FG_OK;
+}
+
+}  // namespace
+
+fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot,
+                              void* out, int32_t n_q_heads, float softmax_scale,
+                              int32_t window, cudaStream_t strm, float* ws, size_t ws_floats,
+                              bool grow_ws);
+
+extern "C" fg_status fg_ragged_attention(const fg_kv_cache* c, fg_ragged_batch* b,
+                                         const void* q_rot, void* out, int32_t n_q_heads,
+                                         float softmax_scale, int32_t sliding_window,
+                                         void* stream) {
+  return fg_attention_launch(c, b, q_rot, out, n_q_heads, softmax_scale, sliding_window,
+                             static_cast<cudaStream_t>(stream), nullptr, 0, true);
+}
+
+// Shared body of the attention entry points. With grow_ws the batch's own
+// workspace is used (and grown); otherwise `ws` / `ws_floats` is.
+fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot,
+                              void* out, int32_t n_q_heads, float softmax_scale,
+                              int32_t window, cudaStream_t strm, float* ws, size_t ws_floats,
+                              bool grow_ws) {
+  fg_status st = check_pass(c, b, n_q_heads);
+  if (st) return st;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(FG_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (window < 0) return fail(FG_ERR_INVALID_ARG, "sliding_window %d < 0", window);
+  if (b->n_tokens == 0) return FG_OK;
+  if (!q_rot || !out) return fail(FG_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q_rot) || !aligned16(out))
+    return fail(FG_ERR_INVALID_ARG, "q_rot and out must be 16-byte aligned");
+  const int32_t g = n_q_heads / c->n_kv_heads;
+  if (g > fg::kMaxGroup)
+    return fail(FG_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads = %d > %d", g, fg::kMaxGroup);
+  st = prepare_plan(b, c, g, window, strm);
+  if (st) return st;
+  const fg::Plan& P = b->plan;
+  const size_t need = (size_t)P.part_rows * (c->head_dim + 2);
+  if (grow_ws) {
+    st = ensure_workspace(b, need, strm);
+    if (st) return st;
+    ws = b->ws;
+  } else if (need > ws_floats) {
+    return fail(FG_ERR_CAPACITY, "pass needs %zu workspace floats, %zu available", need, ws_floats);
+  }
+  float* part_o = ws;
+  float* part_ml = ws ? ws + (size_t)P.part_rows * c->head_dim : nullptr;
+  const float scale_log2 = softmax_scale * 1.4426950408889634f;
+  b->last_launches = (P.n_general > 0) + (P.n_decode > 0) + (P.n_combine > 0);
+  const char* base = static_cast<const char*>(b->dplan);
+  const CacheView cv = cache_view(c);
+  const auto* qr = static_cast<const __nv_bfloat16*>(q_rot);
+  auto* o = static_cast<__nv_bfloat16*>(out);
+  cudaError_t e = fg::launch_attention_general(
+      cv, b->view, reinterpret_cast<const WorkItem*>(base + P.off_general), P.n_general, qr, o,
+      part_o, part_ml, n_q_heads, g, scale_log2, window, strm);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  e = fg::launch_attention_decode(cv, b->view,
+                                  reinterpret_cast<const WorkItem*>(base + P.off_decode), P.n_decode,
+                                  qr, o, part_o, part_ml, n_q_heads, scale_log2, strm);
+  if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
+  e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),
+                         P.n_combine, P.max_combine_rows, part_o, part_ml, o, n_q_heads, g,
+                         c->head_dim, strm);
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  return FG_OK;
+}
+
+extern "C" fg_status fg_attention_plan_info(const fg_ragged_batch* b, int32_t info[8]) {
+  if (!b || !info) return fail(FG_ERR_INVALID_ARG, "NULL argument");
+  const fg::Plan& P = b->plan;
+  info[0] = P.n_general;
+  info[1] = P.n_decode;
+  info[2] = 0;
+  info[3] = P.n_combine;
+  info[4] = P.part_rows;
+  info[5] = b->last_launches;
+  info[6] = info[7] = 0;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_device_status(fg_ragged_batch* b, void* stream) {
+  if (!b) return fail(FG_ERR_INVALID_ARG, "batch is NULL");
+  if (!b->derr) return FG_OK;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  int32_t w = 0;
+  FG_CUDA(cudaMemcpyAsync(&w, b->derr, 4, cudaMemcpyDeviceToHost, strm));
+  FG_CUDA(cudaStreamSynchronize(strm));
+  FG_CUDA(cudaMemsetAsync(b->derr, 0, 4, strm));
+  FG_CUDA(cudaStreamSynchronize(strm));
+  if (w & fg::kErrTimeout) return fail(FG_ERR_TIMEOUT, "a bounded device wait gave up (word 0x%x)", w);
+  if (w) return fail(FG_ERR_DEVICE_CHECK, "a kernel skipped an out-of-range access (word 0x%x)", w);
+  return FG_OK;
+}
+
+extern "C" const char* fg_status_string(fg_status s) {
+  switch (s) {
+    case FG_OK: return "FG_OK";
+    case FG_ERR_INVALID_ARG: return "FG_ERR_INVALID_ARG";
+    case FG_ERR_OUT_OF_RANGE: return "FG_ERR_OUT_OF_RANGE";
+    case FG_ERR_ALIAS: return "FG_ERR_ALIAS";
+    case FG_ERR_CAPACITY: return "FG_ERR_CAPACITY";
+    case FG_ERR_UNSUPPORTED: return "FG_ERR_UNSUPPORTED";
+    case FG_ERR_CUDA: return "FG_ERR_CUDA";
+    case FG_ERR_DEVICE_CHECK: return "FG_ERR_DEVICE_CHECK";
+    case FG_ERR_TIMEOUT: return "FG_ERR_TIMEOUT";
+  }
+  return "FG_ERR_UNKNOWN";
+}
+
+extern "C" const char* fg_last_error(void) { return g_last_error.c_str(); }

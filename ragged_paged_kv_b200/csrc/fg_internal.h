@@ -1,0 +1,90 @@
+// Internal declarations shared by the host library and the CUDA kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace fg {
+
+// Device error word bits (read back by fg_device_status).
+enum : int32_t { kErrBadBlock = 1, kErrBadIndex = 2, kErrTimeout = 4 };
+
+// One attention work unit: the query rows of `n_tok` consecutive new tokens
+// of sequence `seq` (all q heads of kv head `kv_head`), against the cached
+// key positions [key_begin, key_end). Query row r of the unit is token
+// tok_begin + r / g, q head kv_head * g + r % g.
+struct WorkItem {
+  int32_t seq;
+  int32_t kv_head;
+  int32_t tok_begin;  // index within the sequence's new tokens
+  int32_t n_tok;
+  int32_t key_begin;  // absolute position, inclusive
+  int32_t key_end;    // absolute position, exclusive
+  int32_t part;       // -1: write the normalised bf16 output; else first partial row
+  int32_t n_rows;     // n_tok * g
+};
+
+// Rows whose key range was split: `n_splits` partials of n_rows rows each,
+// split i's row r at partial row part_base + i * n_rows + r.
+struct CombineItem {
+  int32_t seq;
+  int32_t kv_head;
+  int32_t tok_begin;
+  int32_t n_tok;
+  int32_t part_base;
+  int32_t n_splits;
+  int32_t n_rows;
+  int32_t pad;
+};
+
+struct CacheView {
+  __nv_bfloat16* base;
+  int32_t n_blocks;
+  int32_t n_kv_heads;
+  int32_t block_size;
+  int32_t head_dim;
+};
+
+struct BatchView {
+  const int32_t* cu_q;     // [S + 1] first batch row of each sequence
+  const int32_t* ctx;      // [S] cached tokens before this pass
+  const int32_t* bt_off;   // [S + 1] CSR offsets into bt
+  const int32_t* bt;       // physical block ids, logical order per sequence
+  const int32_t* tok_seq;  // [T] sequence index of each batch row
+  int32_t n_seqs;
+  int32_t n_tokens;
+  int32_t* err;            // device error word
+};
+
+// Offset in bf16 words of (block, kv, head, slot, dim 0) in the cache.
+__host__ __device__ inline int64_t cache_offset(const CacheView& c, int64_t blk, int kv, int head,
+                                                int slot) {
+  return (((blk * 2 + kv) * c.n_kv_heads + head) * (int64_t)c.block_size + slot) *
+         (int64_t)c.head_dim;
+}
+
+cudaError_t launch_rotary_append(const CacheView& cache, const BatchView& batch,
+                                 const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                 const __nv_bfloat16* v, __nv_bfloat16* q_rot, const float2* rope,
+                                 int n_q_heads, cudaStream_t stream);
+
+cudaError_t launch_attention_general(const CacheView& cache, const BatchView& batch,
+                                     const WorkItem* items, int n_items,
+                                     const __nv_bfloat16* q_rot, __nv_bfloat16* out,
+                                     float* part_o, float* part_ml, int n_q_heads, int g,
+                                     float scale_log2, int window, cudaStream_t stream);
+
+cudaError_t launch_attention_decode(const CacheView& cache, const BatchView& batch,
+                                    const WorkItem* items, int n_items,
+                                    const __nv_bfloat16* q_rot, __nv_bfloat16* out, float* part_o,
+                                    float* part_ml, int n_q_heads, float scale_log2,
+                                    cudaStream_t stream);
+
+cudaError_t launch_combine(const BatchView& batch, const CombineItem* items, int n_items,
+                           int max_rows, const float* part_o, const float* part_ml,
+                           __nv_bfloat16* out, int n_q_heads, int g, int head_dim,
+                           cudaStream_t stream);
+
+}  // namespace fg

@@ -1,0 +1,40 @@
+// Work planning for one ragged attention pass (host, integer work only).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "fg_internal.h"
+
+namespace fg {
+
+constexpr int kMaxGroup = 16;     // q heads per kv head served
+constexpr int kGeneralRows = 16;  // query rows per general-path unit
+constexpr int kSplitKeys = 1024;  // keys per split-KV partial (general path)
+constexpr int kDecodeSplitKeys = 512;  // keys per unit of the MHA decode kernel
+
+struct Plan {
+  std::vector<WorkItem> general;   // CUDA-core general path
+  std::vector<WorkItem> decode;    // one-row MHA decode units (split-KV)
+  std::vector<CombineItem> combine;
+  int32_t part_rows = 0;         // partial rows the split units write
+  int32_t max_combine_rows = 0;  // largest n_rows among combine items
+  // packed device layout (bytes from the plan buffer's start)
+  size_t off_general = 0, off_decode = 0, off_combine = 0, total = 0;
+  int32_t n_general = 0, n_decode = 0, n_combine = 0;
+
+  size_t bytes() const { return total; }
+  void pack(void* dst) const;
+};
+
+// Cut the batch into work units: per sequence and kv head, tiles of new
+// tokens, each over the key range its rows can see (causal, sliding window);
+// long ranges are split into partials merged afterwards by the combine
+// kernel. One-token queries with one q head per kv head go to the decode
+// kernel in kDecodeSplitKeys-key units; everything else to the general path
+// (up to kGeneralRows rows per unit, kSplitKeys keys per partial).
+void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& ctx_lens,
+                int n_kv_heads, int g, int head_dim, int window, Plan* out);
+
+}  // namespace fg

@@ -1,0 +1,264 @@
+"""Python binding of libfg (ctypes). Argument marshalling only: every step of
+the path runs in the library's CUDA kernels; PyTorch supplies device memory
+and streams. If libfg.so is missing this module raises at import of the
+library (there is no fallback of any kind)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfg.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fg.h")
+
+STATUS = {0: "FG_OK", 1: "FG_ERR_INVALID_ARG", 2: "FG_ERR_OUT_OF_RANGE", 3: "FG_ERR_ALIAS",
+          4: "FG_ERR_CAPACITY", 5: "FG_ERR_UNSUPPORTED", 6: "FG_ERR_CUDA",
+          7: "FG_ERR_DEVICE_CHECK", 8: "FG_ERR_TIMEOUT"}
+_c_int32_p = ctypes.POINTER(ctypes.c_int32)
+_c_float_p = ctypes.POINTER(ctypes.c_float)
+
+_lib = None
+
+
+class FgError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        super().__init__(f"{where}: {self.name}: {detail}")
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m ragged_paged_kv_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    V, P, I32, I64, F, D, SZ = (ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32,
+                                ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_size_t)
+    sig = {
+        "fg_kv_cache_create": [I32, I32, I32, I32, P],
+        "fg_kv_cache_create_external": [I32, I32, I32, I32, V, SZ, P],
+        "fg_kv_cache_layout": [V, P, ctypes.POINTER(I64)],
+        "fg_kv_cache_destroy": [V],
+        "fg_ragged_batch_create": [I32, I32, I32, P],
+        "fg_ragged_batch_put": [V, V, I32, _c_int32_p, _c_int32_p, _c_int32_p, _c_int32_p, I32, V],
+        "fg_ragged_batch_shape": [V, _c_int32_p, _c_int32_p],
+        "fg_ragged_batch_destroy": [V],
+        "fg_rotary_kv_append": [V, V, V, V, V, V, I32, D, V],
+        "fg_ragged_attention": [V, V, V, V, I32, F, I32, V],
+        "fg_device_status": [V, V],
+        "fg_attention_plan_info": [V, _c_int32_p],
+        "fg_rotary_table": [D, I32, I32, I32, _c_float_p, _c_float_p],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.fg_status_string.argtypes = [ctypes.c_int]
+    L.fg_status_string.restype = ctypes.c_char_p
+    L.fg_last_error.argtypes = []
+    L.fg_last_error.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise FgError(st, where, lib().fg_last_error().decode())
+
+
+def header_symbols() -> list[str]:
+    """Function names declared in include/fg.h."""
+    txt = open(HEADER_PATH).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(fg_[a-z0-9_]+)\s*\(", txt)))
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    if hasattr(stream, "cuda_stream"):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def _dev_ptr(t, name: str) -> ctypes.c_void_p:
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.element_size() != 2:
+        raise ValueError(f"{name} must hold 16-bit (bf16) elements")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _i32(a, name: str) -> np.ndarray:
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+    return a
+
+
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(_c_int32_p)
+
+
+# ----------------------------------------------------------------------------
+class KVCache:
+    """Blocked KV cache [n_blocks][2][n_kv_heads][block_size][head_dim] bf16.
+
+    By default the pool is a torch tensor (``self.tensor``, viewed as that 5-d
+    shape) registered through fg_kv_cache_create_external, so tests and tools
+    can read and write it; ``owned=True`` lets the library cudaMalloc it."""
+
+    def __init__(self, block_size: int, n_blocks: int, n_kv_heads: int, head_dim: int, *,
+                 tensor=None, owned: bool = False, device=None):
+        import torch
+        self.block_size, self.n_blocks = int(block_size), int(n_blocks)
+        self.n_kv_heads, self.head_dim = int(n_kv_heads), int(head_dim)
+        self._h = ctypes.c_void_p()
+        self.tensor = None
+        if owned:
+            _check(lib().fg_kv_cache_create(self.block_size, self.n_blocks, self.n_kv_heads,
+                                            self.head_dim, ctypes.byref(self._h)),
+                   "fg_kv_cache_create")
+            return
+        shape = (self.n_blocks, 2, self.n_kv_heads, self.block_size, self.head_dim)
+        if tensor is None:
+            tensor = torch.empty(shape, dtype=torch.bfloat16, device=device or "cuda")
+        if tuple(tensor.shape) != shape:
+            raise ValueError(f"cache tensor shape {tuple(tensor.shape)} != {shape}")
+        self.tensor = tensor
+        _check(lib().fg_kv_cache_create_external(self.block_size, self.n_blocks, self.n_kv_heads,
+                                                 self.head_dim, _dev_ptr(tensor, "cache"),
+                                                 tensor.numel() * 2, ctypes.byref(self._h)),
+               "fg_kv_cache_create_external")
+
+    @property
+    def handle(self):
+        return self._h
+
+    def layout(self):
+        base = ctypes.c_void_p()
+        strides = (ctypes.c_int64 * 5)()
+        _check(lib().fg_kv_cache_layout(self._h, ctypes.byref(base), strides), "fg_kv_cache_layout")
+        return base.value, list(strides)
+
+    def close(self):
+        if self._h:
+            lib().fg_kv_cache_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class RaggedBatch:
+    """Holder of one pass's batch metadata (fg_ragged_batch)."""
+
+    def __init__(self, max_tokens: int, max_seqs: int, max_blocks_per_seq: int):
+        self._h = ctypes.c_void_p()
+        self.max_tokens, self.max_seqs, self.max_blocks_per_seq = max_tokens, max_seqs, max_blocks_per_seq
+        _check(lib().fg_ragged_batch_create(int(max_tokens), int(max_seqs), int(max_blocks_per_seq),
+                                            ctypes.byref(self._h)), "fg_ragged_batch_create")
+
+    @property
+    def handle(self):
+        return self._h
+
+    def put(self, cache: KVCache, seq_ids, q_lens, ctx_lens, block_tables, stream=None):
+        ids, ql, cl = _i32(seq_ids, "seq_ids"), _i32(q_lens, "q_lens"), _i32(ctx_lens, "ctx_lens")
+        bt = _i32(block_tables, "block_tables")
+        if bt.ndim != 2:
+            raise ValueError("block_tables must be 2-d [n_seqs, stride]")
+        n = len(ql)
+        if not (len(ids) == len(cl) == n == bt.shape[0]):
+            raise ValueError("seq_ids, q_lens, ctx_lens and block_tables rows must agree")
+        st = _stream_ptr(stream) if n else ctypes.c_void_p(0)
+        _check(lib().fg_ragged_batch_put(self._h, cache.handle, n, _i32p(ids), _i32p(ql), _i32p(cl),
+                                         _i32p(bt), int(bt.shape[1]) if n else 1, st),
+               "fg_ragged_batch_put")
+
+    def shape(self):
+        t, s = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().fg_ragged_batch_shape(self._h, ctypes.byref(t), ctypes.byref(s)), "fg_ragged_batch_shape")
+        return t.value, s.value
+
+    def plan_info(self) -> dict:
+        a = (ctypes.c_int32 * 8)()
+        _check(lib().fg_attention_plan_info(self._h, ctypes.cast(a, _c_int32_p)), "fg_attention_plan_info")
+        keys = ("general_units", "decode_units", "tensor_units", "combine_groups", "partial_rows",
+                "launches")
+        return dict(zip(keys, list(a)[:6]))
+
+    def device_status(self, stream=None):
+        _check(lib().fg_device_status(self._h, _stream_ptr(stream)), "fg_device_status")
+
+    def close(self):
+        if self._h:
+            lib().fg_ragged_batch_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def rotary_kv_append(cache: KVCache, batch: RaggedBatch, q, k, v, q_rot, n_q_heads: int,
+                     rope_theta: float, stream=None):
+    _check(lib().fg_rotary_kv_append(cache.handle, batch.handle, _dev_ptr(q, "q"), _dev_ptr(k, "k"),
+                                     _dev_ptr(v, "v"), _dev_ptr(q_rot, "q_rot"), int(n_q_heads),
+                                     float(rope_theta), _stream_ptr(stream)),
+           "fg_rotary_kv_append")
+
+
+def ragged_attention(cache: KVCache, batch: RaggedBatch, q_rot, out, n_q_heads: int,
+                     softmax_scale: float, sliding_window: int = 0, stream=None):
+    _check(lib().fg_ragged_attention(cache.handle, batch.handle, _dev_ptr(q_rot, "q_rot"),
+                                     _dev_ptr(out, "out"), int(n_q_heads), float(softmax_scale),
+                                     int(sliding_window), _stream_ptr(stream)),
+           "fg_ragged_attention")
+
+
+def rotary_table(rope_theta: float, head_dim: int, pos_begin: int, n_pos: int):
+    """Host float32 cos/sin tables [n_pos, head_dim/2] exactly as libfg builds them."""
+    c = np.empty((n_pos, head_dim // 2), np.float32)
+    s = np.empty((n_pos, head_dim // 2), np.float32)
+    _check(lib().fg_rotary_table(float(rope_theta), int(head_dim), int(pos_begin), int(n_pos),
+                                 c.ctypes.data_as(_c_float_p), s.ctypes.data_as(_c_float_p)),
+           "fg_rotary_table")
+    return c, s
+
+
+def forward(cache: KVCache, batch: RaggedBatch, q, k, v, q_rot, out, n_q_heads: int,
+            rope_theta: float, softmax_scale: float, sliding_window: int = 0, stream=None):
+    """One pass on device tensors: rotary + append, then ragged attention."""
+    rotary_kv_append(cache, batch, q, k, v, q_rot, n_q_heads, rope_theta, stream)
+    ragged_attention(cache, batch, q_rot, out, n_q_heads, softmax_scale, sliding_window, stream)
+
+
+def forward_host(cache: KVCache, batch: RaggedBatch, host_in: dict, dev: dict, host_out,
+                 n_q_heads: int, rope_theta: float, softmax_scale: float,
+                 sliding_window: int = 0, stream=None):
+    """One pass from host buffers: pinned host q/k/v (``host_in``) are copied to
+    the device tensors in ``dev`` ('q', 'k', 'v', 'q_rot', 'out'), the pass runs,
+    and the output is copied back into pinned ``host_out``; all on ``stream``."""
+    import torch
+    s = stream or torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        for name in ("q", "k", "v"):
+            dev[name].copy_(host_in[name], non_blocking=True)
+        forward(cache, batch, dev["q"], dev["k"], dev["v"], dev["q_rot"], dev["out"], n_q_heads,
+                rope_theta, softmax_scale, sliding_window, s)
+        host_out.copy_(dev["out"], non_blocking=True)

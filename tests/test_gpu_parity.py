@@ -1,0 +1,245 @@
+"""GPU path vs the float64 oracle, through the C ABI.
+
+Bars: rotated Q and every word of the cache blocks a checked sequence owns
+(new tokens, prior context and untouched slots alike) bit-exact; attention
+outputs within max-abs 2e-2 and relative L2 5e-3 (bf16 operands, fp32
+accumulation). Full-size workloads are checked on sampled sequences and
+tokens the oracle computes one by one; small ones on every output."""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import PagedCache
+from oracle.forward import splitfuse_pass
+from ragged_paged_kv_b200 import fg, fixtures
+from ragged_paged_kv_b200 import workloads as W
+from ragged_paged_kv_b200.fixtures import SENTINEL, to_bits
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, REL_L2 = 2e-2, 5e-3
+
+
+def assert_close(got, ref, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err.max() <= MAX_ABS and rel <= REL_L2, f"{what}: max-abs {err.max():.3g}, rel-L2 {rel:.3g}"
+
+
+def bf16_to_f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def run_gpu(w, keep, cache=None, fill=True, write_ctx=True, inplace=False, others="random"):
+    if cache is None:
+        cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+        if fill:
+            fixtures.fill(cache.tensor)
+    kept = fixtures.write_context(w, cache.tensor, set(keep), others=others) if write_ctx else {}
+    batch = fg.RaggedBatch(max(w.n_tokens, 1), max(w.n_seqs, 1), max(w.block_tables.shape[1], 1))
+    batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables)
+    q, k, v = fixtures.qkv_device(w)
+    q_rot = q if inplace else torch.empty_like(q)
+    out = torch.full_like(q, float("nan"))
+    fg.forward(cache, batch, q, k, v, q_rot, out, w.n_q_heads, w.rope_theta, w.softmax_scale,
+               w.sliding_window)
+    torch.cuda.synchronize()
+    batch.device_status()
+    return cache, batch, q_rot, out, kept
+
+
+def run_oracle(w, kept, tokens=None, pc=None):
+    if pc is None:
+        pc = PagedCache(w.n_blocks, w.n_kv_heads, w.block_size, w.head_dim, fill=SENTINEL)
+        for s, (ids, blocks) in kept.items():
+            for i, b in enumerate(ids):
+                pc.blocks[int(b)] = blocks[i].copy()
+    q, k, v = w.qkv()
+    q_rot, _, out = splitfuse_pass(pc, w.block_tables, w.q_lens, w.ctx_lens, q, k, v,
+                                   w.rope_theta, w.softmax_scale, w.sliding_window, tokens)
+    return pc, q_rot, out
+
+
+def sample_tokens(w, seqs, per_seq=48, seed=0):
+    rng = np.random.default_rng(seed)
+    cu = w.cu_q
+    toks = []
+    for s in seqs:
+        a, b = int(cu[s]), int(cu[s + 1])
+        if b - a <= per_seq:
+            toks.extend(range(a, b))
+        else:
+            mid = rng.choice(np.arange(a + 8, b - 8), per_seq - 16, replace=False)
+            toks.extend(list(range(a, a + 8)) + sorted(mid.tolist()) + list(range(b - 8, b)))
+    return np.array(sorted(set(toks)), dtype=np.int64)
+
+
+def check_pass(w, keep, per_seq=48, check_cache=True, others="random"):
+    cache, batch, q_rot, out, kept = run_gpu(w, keep, others=others)
+    tokens = sample_tokens(w, keep, per_seq)
+    pc, q_rot_ref, ref = run_oracle(w, kept, tokens)
+    assert np.array_equal(to_bits(q_rot), q_rot_ref), "rotated Q differs"
+    if check_cache:
+        for s in keep:
+            ids = w.block_tables[s, :w.blocks_used(s)].astype(np.int64)
+            dev = to_bits(cache.tensor[torch.from_numpy(ids).cuda()])
+            for i, b in enumerate(ids):
+                assert np.array_equal(dev[i], pc.block(int(b))), f"cache block {b} of seq {s} differs"
+    all_out = to_bits(out)
+    assert np.isfinite(bf16_to_f64(all_out)).all(), "non-finite output somewhere in the batch"
+    got = bf16_to_f64(all_out[tokens])
+    assert_close(got, ref[tokens], w.name)
+    return cache, out
+
+
+def _free(*objs):
+    for o in objs:
+        if hasattr(o, "close"):
+            o.close()
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def test_config1_tiny_every_output():
+    w = W.config1()
+    cache, out = check_pass(w, keep=range(w.n_seqs), per_seq=1000)
+    # blocks outside every table are untouched
+    used = set(np.concatenate([w.block_tables[s, :w.blocks_used(s)] for s in range(w.n_seqs)]).tolist())
+    free_ids = [b for b in range(w.n_blocks) if b not in used]
+    assert (to_bits(cache.tensor[free_ids]) == SENTINEL).all()
+    _free(cache)
+
+
+def test_config2_llama7b_splitfuse_snapshot():
+    w = W.config2()
+    keep = list(range(w.n_seqs))
+    cache, _ = check_pass(w, keep, per_seq=96)
+    _free(cache)
+
+
+def test_config3_decode_heavy_large_pool():
+    free, _ = torch.cuda.mem_get_info()
+    B = 2 * 32 * 64 * 128 * 2
+    n_blocks = int(min(180 * 10**9, free - 8 * 2**30) // B)
+    w = W.config3(n_blocks=n_blocks)
+    keep = sorted(np.random.default_rng(3).choice(w.n_seqs, 24, replace=False).tolist())
+    cache, _ = check_pass(w, keep, others="pool")
+    _free(cache)
+
+
+def test_config4_mistral_gqa_window():
+    w = W.config4()
+    rng = np.random.default_rng(4)
+    keep = [0, 1, 2, 3] + sorted(rng.choice(np.arange(4, w.n_seqs), 48, replace=False).tolist())
+    cache, _ = check_pass(w, keep, per_seq=64)
+    _free(cache)
+
+
+def test_config5_llama70b_long_prompt():
+    w = W.config5()
+    rng = np.random.default_rng(5)
+    keep = [0] + sorted(rng.choice(np.arange(1, w.n_seqs), 12, replace=False).tolist())
+    cache, _ = check_pass(w, keep, per_seq=48)
+    _free(cache)
+
+
+def test_block_permutation_gives_bit_identical_output():
+    for w in (W.config1(), W.config2()):
+        c1, b1, _, o1, _ = run_gpu(w, keep=())
+        r1 = to_bits(o1)
+        _free(c1, b1)
+        w2 = w.with_permuted_blocks(7)
+        c2, b2, _, o2, _ = run_gpu(w2, keep=())
+        assert np.array_equal(r1, to_bits(o2)), w.name
+        _free(c2, b2)
+
+
+def test_window_covering_everything_equals_no_window():
+    w = W.config1()
+    c1, b1, _, o1, _ = run_gpu(w, keep=())
+    w.sliding_window = 1 << 20
+    c2, b2, _, o2, _ = run_gpu(w, keep=())
+    assert np.array_equal(to_bits(o1), to_bits(o2))
+    _free(c1, b1, c2, b2)
+
+
+def test_in_place_rotation_matches_out_of_place():
+    w = W.config1()
+    c1, b1, qr1, o1, _ = run_gpu(w, keep=())
+    c2, b2, qr2, o2, _ = run_gpu(w, keep=(), inplace=True)
+    assert np.array_equal(to_bits(qr1), to_bits(qr2)) and np.array_equal(to_bits(o1), to_bits(o2))
+    _free(c1, b1, c2, b2)
+
+
+def test_empty_batch_is_a_no_op():
+    cache = fg.KVCache(16, 8, 2, 64)
+    fixtures.fill(cache.tensor)
+    batch = fg.RaggedBatch(4, 2, 2)
+    batch.put(cache, [], [], [], np.zeros((0, 1), np.int32))
+    z = torch.empty((0, 4, 64), dtype=torch.bfloat16, device="cuda")
+    fg.forward(cache, batch, z, z[:, :2], z[:, :2], z, z, 4, 1e4, 0.125)
+    torch.cuda.synchronize()
+    batch.device_status()
+    assert batch.shape() == (0, 0)
+    assert (to_bits(cache.tensor) == SENTINEL).all()
+    _free(cache, batch)
+
+
+@pytest.mark.parametrize("B,d,Hq,Hkv,window", [
+    (16, 64, 4, 4, 0), (32, 128, 8, 2, 0), (64, 128, 8, 1, 0), (128, 64, 6, 3, 0),
+    (16, 128, 16, 2, 37), (64, 64, 4, 4, 300), (128, 128, 32, 8, 0), (32, 64, 16, 16, 1)])
+def test_shape_sweep(B, d, Hq, Hkv, window):
+    """Ragged tails everywhere: lengths off every tile / block / stage size."""
+    rng = np.random.default_rng(B * 7 + d + Hq * 3 + Hkv + window)
+    q_lens = [1, 1, 3, 130, 17, 1, 257]
+    ctx_lens = [0, 700, 64, 0, 1111, 2049, 90]
+    w = W._make(f"sweep_B{B}_d{d}_g{Hq // Hkv}_w{window}", Hq, Hkv, d, B, list(range(7)),
+                q_lens, ctx_lens, seed=int(rng.integers(1 << 30)), budget=sum(q_lens),
+                window=window)
+    keep = list(range(w.n_seqs))
+    cache, _ = check_pass(w, keep, per_seq=1000)
+    _free(cache)
+
+
+def test_chunked_prefill_equals_one_shot_70b_shape():
+    """One 32768-token prompt (64/8 heads): 16 chunks of 2048 through the API
+    build the same cache bits as the one-shot pass; outputs agree within
+    tolerance with each other and with the oracle on sampled rows."""
+    one = W.prompt_chunks(64, 8, 128, 64, 32768, 32768, seed=55)[0]
+    chunks = W.prompt_chunks(64, 8, 128, 64, 32768, 2048, seed=55)
+    ids = torch.from_numpy(one.block_tables[0].astype(np.int64)).cuda()
+    c1, b1, _, o1, _ = run_gpu(one, keep=(), write_ctx=False)
+    blocks1 = to_bits(c1.tensor[ids])
+    out1 = to_bits(o1)
+    _free(b1)
+    del o1
+    c2 = fg.KVCache(64, one.n_blocks, 8, 128)
+    fixtures.fill(c2.tensor)
+    outs = []
+    for w in chunks:
+        _, b2, _, o2, _ = run_gpu(w, keep=(), cache=c2, write_ctx=False)
+        outs.append(to_bits(o2))
+        _free(b2)
+    assert np.array_equal(to_bits(c2.tensor[ids]), blocks1)
+    out2 = np.concatenate(outs)
+    assert_close(bf16_to_f64(out2), bf16_to_f64(out1), "chunked vs one-shot")
+    # oracle on sampled rows of the one-shot pass
+    pc = PagedCache(one.n_blocks, 8, 64, 128, fill=SENTINEL)
+    for i, b in enumerate(one.block_tables[0]):
+        pc.blocks[int(b)] = blocks1[i].copy()
+    from oracle import attention, rotary
+    q, _, _ = one.qkv()
+    tok = np.sort(np.random.default_rng(1).choice(32768, 24, replace=False))
+    tok = np.unique(np.concatenate([tok, [0, 1, 2047, 2048, 32767]]))
+    q_rot = rotary.rotate_half(q[tok], tok, 1e4)
+    ref = np.full(q.shape, np.nan)
+    for i, p in enumerate(tok):      # each sampled row as a one-token pass at its position
+        ref[p] = attention.ragged_attention(pc, one.block_tables, [1], [int(p)], q_rot[i:i + 1],
+                                            one.softmax_scale)[0]
+    assert_close(bf16_to_f64(out1[tok]), ref[tok], "one-shot vs oracle")
+    _free(c1, c2)
