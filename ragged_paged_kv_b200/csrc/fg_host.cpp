@@ -13,6 +13,9 @@
 #include <string>
 #include <vector>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "../../include/fg.h"
 #include "fg_internal.h"
 #include "fg_plan.h"
@@ -112,6 +115,9 @@ struct fg_kv_cache {
   double rope_theta = 0.0;
   int32_t rope_npos = 0;
   float2* rope = nullptr;
+  // TMA view of the pool: 2-D (head_dim, every slot row), 64 x min(B, 64) boxes
+  alignas(64) CUtensorMap tm_kv;
+  int tm_kv_state = 0;  // 0 = not built, 1 = built, -1 = unavailable
 };
 
 struct fg_ragged_batch {
@@ -520,13 +526,70 @@ extern "C" fg_status fg_rotary_kv_append(fg_kv_cache* c, const fg_ragged_batch* 
 
 namespace {
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda). nullptr if the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// The pool as a 2-D bf16 tensor: inner dim head_dim, outer dim every slot row
+// ((block * 2 + kv) * Hkv + head) * B + slot; boxes of 64 dims x min(B, 64)
+// rows, 128-byte swizzle (the layout the tensor-core operands use).
+bool ensure_kv_map(fg_kv_cache* c) {
+  if (c->tm_kv_state) return c->tm_kv_state > 0;
+  c->tm_kv_state = -1;
+  auto enc = tensor_map_encoder();
+  const uint64_t rows = (uint64_t)c->n_blocks * 2 * c->n_kv_heads * c->block_size;
+  if (!enc || rows >= (1ull << 31)) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)c->head_dim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)c->head_dim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)std::min(c->block_size, 64)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&c->tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c->base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  c->tm_kv_state = 1;
+  return true;
+}
+
+// q_rot as a 3-D bf16 tensor (head_dim, n_q_heads, tokens); a box of
+// 64 dims x g heads x 128/g tokens lands as 128 rows (token-major, head-minor)
+// of 128 bytes, the A-operand layout of a query tile.
+bool make_q_map(CUtensorMap* m, const void* q_rot, int T, int Hq, int d, int g) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)Hq, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)Hq * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)g, (cuuint32_t)(fg::kTcRows / g)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q_rot), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tc_eligible(fg_kv_cache* c, int g) {
+  const bool pow2 = g >= 1 && g <= fg::kTcRows && (g & (g - 1)) == 0;
+  return pow2 && ensure_kv_map(c);
+}
+
 // Upload the plan for (g, window) unless the batch's current plan already is.
 fg_status prepare_plan(fg_ragged_batch* b, const fg_kv_cache* c, int32_t g, int32_t window,
-                       cudaStream_t strm) {
+                       bool use_tc, cudaStream_t strm) {
   const uint64_t key[4] = {b->put_gen, (uint64_t)g, (uint64_t)(uint32_t)window,
-                           (uint64_t)c->head_dim};
+                           (uint64_t)c->head_dim | ((uint64_t)use_tc << 32)};
   if (std::equal(key, key + 4, b->plan_key) && b->dplan) return FG_OK;
-  fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, &b->plan);
+  fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc, &b->plan);
   const size_t bytes = b->plan.bytes();
   if (bytes > b->dplan_bytes) {
     if (b->dplan) FG_CUDA(cudaFreeAsync(b->dplan, strm));
@@ -590,9 +653,13 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   if (!aligned16(q_rot) || !aligned16(out))
     return fail(FG_ERR_INVALID_ARG, "q_rot and out must be 16-byte aligned");
   const int32_t g = n_q_heads / c->n_kv_heads;
-  if (g > fg::kMaxGroup)
+  const bool use_tc = tc_eligible(const_cast<fg_kv_cache*>(c), g);
+  if (!use_tc && g > fg::kMaxGroup)
     return fail(FG_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads = %d > %d", g, fg::kMaxGroup);
-  st = prepare_plan(b, c, g, window, strm);
+  CUtensorMap tm_q;
+  if (use_tc && !make_q_map(&tm_q, q_rot, b->n_tokens, n_q_heads, c->head_dim, g))
+    return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q_rot");
+  st = prepare_plan(b, c, g, window, use_tc, strm);
   if (st) return st;
   const fg::Plan& P = b->plan;
   const size_t need = (size_t)P.part_rows * (c->head_dim + 2);
@@ -606,7 +673,7 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   float* part_o = ws;
   float* part_ml = ws ? ws + (size_t)P.part_rows * c->head_dim : nullptr;
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
-  b->last_launches = (P.n_general > 0) + (P.n_decode > 0) + (P.n_combine > 0);
+  b->last_launches = (P.n_general > 0) + (P.n_decode > 0) + (P.n_tc > 0) + (P.n_combine > 0);
   const char* base = static_cast<const char*>(b->dplan);
   const CacheView cv = cache_view(c);
   const auto* qr = static_cast<const __nv_bfloat16*>(q_rot);
@@ -619,6 +686,12 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
                                   reinterpret_cast<const WorkItem*>(base + P.off_decode), P.n_decode,
                                   qr, o, part_o, part_ml, n_q_heads, scale_log2, strm);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
+  if (P.n_tc) {
+    e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
+                                reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
+                                part_ml, n_q_heads, g, scale_log2, window, strm);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
+  }
   e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),
                          P.n_combine, P.max_combine_rows, part_o, part_ml, o, n_q_heads, g,
                          c->head_dim, strm);
@@ -631,7 +704,7 @@ extern "C" fg_status fg_attention_plan_info(const fg_ragged_batch* b, int32_t in
   const fg::Plan& P = b->plan;
   info[0] = P.n_general;
   info[1] = P.n_decode;
-  info[2] = 0;
+  info[2] = P.n_tc;
   info[3] = P.n_combine;
   info[4] = P.part_rows;
   info[5] = b->last_launches;

@@ -82,6 +82,12 @@ cudaError_t launch_attention_decode(const CacheView& cache, const BatchView& bat
                                     float* part_ml, int n_q_heads, float scale_log2,
                                     cudaStream_t stream);
 
+// tm_q / tm_kv point to CUtensorMap objects (host memory, passed by value).
+cudaError_t launch_attention_tc(const void* tm_q, const void* tm_kv, const CacheView& cache,
+                                const BatchView& batch, const WorkItem* items, int n_items,
+                                __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
+                                int g, float scale_log2, int window, cudaStream_t stream);
+
 cudaError_t launch_combine(const BatchView& batch, const CombineItem* items, int n_items,
                            int max_rows, const float* part_o, const float* part_ml,
                            __nv_bfloat16* out, int n_q_heads, int g, int head_dim,

@@ -11,15 +11,17 @@ void Plan::pack(void* dst) const {
   char* p = static_cast<char*>(dst);
   if (n_general) std::memcpy(p + off_general, general.data(), general.size() * sizeof(WorkItem));
   if (n_decode) std::memcpy(p + off_decode, decode.data(), decode.size() * sizeof(WorkItem));
+  if (n_tc) std::memcpy(p + off_tc, tc.data(), tc.size() * sizeof(WorkItem));
   if (n_combine) std::memcpy(p + off_combine, combine.data(), combine.size() * sizeof(CombineItem));
 }
 
 void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& ctx_lens,
-                int n_kv_heads, int g, int head_dim, int window, Plan* out) {
+                int n_kv_heads, int g, int head_dim, int window, bool use_tc, Plan* out) {
   (void)head_dim;
   Plan& P = *out;
   P.general.clear();
   P.decode.clear();
+  P.tc.clear();
   P.combine.clear();
   P.part_rows = 0;
   P.max_combine_rows = 0;
@@ -53,6 +55,17 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
       for (int h = 0; h < n_kv_heads; ++h) emit(P.decode, s, h, 0, 1, kb, c + 1, kDecodeSplitKeys);
       continue;
     }
+    if (use_tc) {
+      const int tpt = kTcRows / g;
+      for (int t0 = 0; t0 < q; t0 += tpt) {
+        const int nt = std::min(tpt, q - t0);
+        const int p0 = c + t0, p1 = c + t0 + nt - 1;
+        const int kb = window > 0 ? std::max(0, p0 - window + 1) : 0;
+        const int split = nt * g <= 16 ? kTcDecodeSplitKeys : (1 << 30);
+        for (int h = 0; h < n_kv_heads; ++h) emit(P.tc, s, h, t0, nt, kb, p1 + 1, split);
+      }
+      continue;
+    }
     for (int t0 = 0; t0 < q; t0 += tok_per_tile) {
       const int nt = std::min(tok_per_tile, q - t0);
       const int p0 = c + t0, p1 = c + t0 + nt - 1;
@@ -64,12 +77,17 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
   std::stable_sort(P.decode.begin(), P.decode.end(), [](const WorkItem& a, const WorkItem& b) {
     return a.key_end - a.key_begin > b.key_end - b.key_begin;
   });
+  std::stable_sort(P.tc.begin(), P.tc.end(), [](const WorkItem& a, const WorkItem& b) {
+    return a.key_end - a.key_begin > b.key_end - b.key_begin;
+  });
   P.n_general = (int32_t)P.general.size();
   P.n_decode = (int32_t)P.decode.size();
+  P.n_tc = (int32_t)P.tc.size();
   P.n_combine = (int32_t)P.combine.size();
   P.off_general = 0;
   P.off_decode = align_up(P.general.size() * sizeof(WorkItem), 256);
-  P.off_combine = align_up(P.off_decode + P.decode.size() * sizeof(WorkItem), 256);
+  P.off_tc = align_up(P.off_decode + P.decode.size() * sizeof(WorkItem), 256);
+  P.off_combine = align_up(P.off_tc + P.tc.size() * sizeof(WorkItem), 256);
   P.total = align_up(P.off_combine + P.combine.size() * sizeof(CombineItem), 256);
 }
 
