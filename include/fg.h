@@ -164,6 +164,33 @@ fg_status fg_ragged_attention(const fg_kv_cache* cache, fg_ragged_batch* batch, 
                               void* out, int32_t n_q_heads, float softmax_scale,
                               int32_t sliding_window, void* stream);
 
+/* The same pass as fg_ragged_attention, for callers that must not allocate.
+ * The pages have no counterpart: this is a library convenience. Some callers
+ * cannot call cudaMalloc (or cudaMallocAsync / cudaFree, or a framework
+ * allocator) when the pass runs: a server that reserved all of HBM for the KV
+ * pool up front, code under an allocation policy that forbids device
+ * allocation inside a step, or a host framework that owns device memory
+ * itself. This entry point allocates nothing, on the device or pinned on the
+ * host. Its split-KV workspace and its work plan live in two fixed arrays in
+ * the library's device image (8 Mi floats = 32 MiB and 4 MiB), which every
+ * GPU that loads the library holds until the process exits.
+ *   - Limits: a pass whose split partials need more than 8 Mi floats
+ *     (partial rows * (head_dim + 2)) or whose work plan exceeds 4 MiB
+ *     returns FG_ERR_CAPACITY before any launch.
+ *   - First use on a device: the call looks up the arrays' device addresses
+ *     (cudaGetSymbolAddress, with that device current). Make that first call
+ *     before any stream capture.
+ *   - The plan is sent with a copy from ordinary (pageable) host memory, so
+ *     the call may wait for work already queued on `stream`.
+ *   - The arrays are shared by every call in the process and keep the last
+ *     call's contents; nothing in them needs to start at zero (each call
+ *     writes every value it reads). Calls whose device work overlaps (two
+ *     streams, or two threads) race on the arrays: serialise them.
+ * Arguments, layouts and errors are those of fg_ragged_attention. */
+fg_status fg_ragged_attention_noalloc(const fg_kv_cache* cache, fg_ragged_batch* batch,
+                                      const void* q_rot, void* out, int32_t n_q_heads,
+                                      float softmax_scale, int32_t sliding_window, void* stream);
+
 /* Work plan of the batch's last fg_ragged_attention call, for profiling:
  * info[0] = general-path units, info[1] = split-KV decode units,
  * info[2] = tensor-core units, info[3] = combine groups, info[4] = partial

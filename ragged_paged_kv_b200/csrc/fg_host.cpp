@@ -742,3 +742,72 @@ extern "C" const char* fg_status_string(fg_status s) {
 }
 
 extern "C" const char* fg_last_error(void) { return g_last_error.c_str(); }
+
+// Attention pass on caller-provided device storage: the split workspace is
+// `ws` (ws_floats floats) and the work plan is uploaded into `plan_dev`
+// (plan_bytes bytes) with a plain copy from host memory. Nothing is
+// allocated on the device or pinned on the host. The batch's own plan cache
+// and workspace are left alone.
+fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot,
+                                    void* out, int32_t n_q_heads, float softmax_scale,
+                                    int32_t window, cudaStream_t strm, float* ws,
+                                    size_t ws_floats, void* plan_dev, size_t plan_bytes) {
+  fg_status st = check_pass(c, b, n_q_heads);
+  if (st) return st;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(FG_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (window < 0) return fail(FG_ERR_INVALID_ARG, "sliding_window %d < 0", window);
+  if (b->n_tokens == 0) return FG_OK;
+  if (!q_rot || !out) return fail(FG_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q_rot) || !aligned16(out))
+    return fail(FG_ERR_INVALID_ARG, "q_rot and out must be 16-byte aligned");
+  const int32_t g = n_q_heads / c->n_kv_heads;
+  const bool use_tc = tc_eligible(const_cast<fg_kv_cache*>(c), g);
+  if (!use_tc && g > fg::kMaxGroup)
+    return fail(FG_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads = %d > %d", g, fg::kMaxGroup);
+  CUtensorMap tm_q;
+  if (use_tc && !make_q_map(&tm_q, q_rot, b->n_tokens, n_q_heads, c->head_dim, g))
+    return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q_rot");
+  thread_local fg::Plan P;
+  thread_local std::vector<unsigned char> packed;
+  fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc, &P);
+  if (P.bytes() > plan_bytes)
+    return fail(FG_ERR_CAPACITY, "pass needs a %zu-byte work plan, the fixed area holds %zu",
+                P.bytes(), plan_bytes);
+  const size_t need = (size_t)P.part_rows * (c->head_dim + 2);
+  if (need > ws_floats)
+    return fail(FG_ERR_CAPACITY, "pass needs %zu split-workspace floats, the fixed area holds %zu",
+                need, ws_floats);
+  packed.resize(P.bytes());
+  P.pack(packed.data());
+  if (!packed.empty())
+    FG_CUDA(cudaMemcpyAsync(plan_dev, packed.data(), packed.size(), cudaMemcpyHostToDevice, strm));
+  float* part_o = ws;
+  float* part_ml = ws + (size_t)P.part_rows * c->head_dim;
+  const float scale_log2 = softmax_scale * 1.4426950408889634f;
+  const char* base = static_cast<const char*>(plan_dev);
+  const CacheView cv = cache_view(c);
+  const auto* qr = static_cast<const __nv_bfloat16*>(q_rot);
+  auto* o = static_cast<__nv_bfloat16*>(out);
+  cudaError_t e = fg::launch_attention_general(
+      cv, b->view, reinterpret_cast<const WorkItem*>(base + P.off_general), P.n_general, qr, o,
+      part_o, part_ml, n_q_heads, g, scale_log2, window, strm);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  e = fg::launch_attention_decode(cv, b->view, reinterpret_cast<const WorkItem*>(base + P.off_decode),
+                                  P.n_decode, qr, o, part_o, part_ml, n_q_heads, scale_log2, strm);
+  if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
+  if (P.n_tc) {
+    e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
+                                reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
+                                part_ml, n_q_heads, g, scale_log2, window, strm);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
+  }
+  e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),
+                         P.n_combine, P.max_combine_rows, part_o, part_ml, o, n_q_heads, g,
+                         c->head_dim, strm);
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  return FG_OK;
+}
+
+// Sets the thread-local error text (for entry points defined in other files).
+fg_status fg_set_error(fg_status st, const char* msg) { return fail(st, "%s", msg); }

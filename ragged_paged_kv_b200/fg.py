@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
         "fg_ragged_batch_destroy": [V],
         "fg_rotary_kv_append": [V, V, V, V, V, V, I32, D, V],
         "fg_ragged_attention": [V, V, V, V, I32, F, I32, V],
+        "fg_ragged_attention_noalloc": [V, V, V, V, I32, F, I32, V],
         "fg_device_status": [V, V],
         "fg_attention_plan_info": [V, _c_int32_p],
         "fg_rotary_table": [D, I32, I32, I32, _c_float_p, _c_float_p],
@@ -229,6 +230,16 @@ def ragged_attention(cache: KVCache, batch: RaggedBatch, q_rot, out, n_q_heads: 
                                      _dev_ptr(out, "out"), int(n_q_heads), float(softmax_scale),
                                      int(sliding_window), _stream_ptr(stream)),
            "fg_ragged_attention")
+
+
+def ragged_attention_noalloc(cache: KVCache, batch: RaggedBatch, q_rot, out, n_q_heads: int,
+                             softmax_scale: float, sliding_window: int = 0, stream=None):
+    """fg_ragged_attention_noalloc: the attention pass for callers that cannot
+    allocate; uses the library's fixed device arrays (see include/fg.h)."""
+    _check(lib().fg_ragged_attention_noalloc(cache.handle, batch.handle, _dev_ptr(q_rot, "q_rot"),
+                                             _dev_ptr(out, "out"), int(n_q_heads), float(softmax_scale),
+                                             int(sliding_window), _stream_ptr(stream)),
+           "fg_ragged_attention_noalloc")
 
 
 def rotary_table(rope_theta: float, head_dim: int, pos_begin: int, n_pos: int):
