@@ -82,19 +82,40 @@ def algorithmic_work(w):
     append bytes: new K, V read and written to the cache, Q read, Q_rot written.
     flops: 4 * d * Hq per admitted (query, key) pair (QK^T and PV)."""
     Hq, Hkv, d, W = w.n_q_heads, w.n_kv_heads, w.head_dim, w.sliding_window
-    kv_rows = 0
-    pairs = 0
+    g = Hq // Hkv
+    kv_rows = pairs = 0
+    dec_rows = dec_tokens = 0      # one-token MHA decodes: the split-KV decode kernel
+    tc_pairs = tc_rows = 0         # everything else: the tensor-core kernel
     for q, c in zip(w.q_lens.tolist(), w.ctx_lens.tolist()):
         p = np.arange(c, c + q, dtype=np.int64)
         lo = np.maximum(0, p - W + 1) if W > 0 else np.zeros_like(p)
-        kv_rows += int(p[-1] + 1 - lo[0])
-        pairs += int((p - lo + 1).sum())
+        rows = int(p[-1] + 1 - lo[0])
+        prs = int((p - lo + 1).sum())
+        kv_rows += rows
+        pairs += prs
+        if q == 1 and g == 1:
+            dec_rows += rows
+            dec_tokens += 1
+        else:
+            tc_rows += rows
+            tc_pairs += prs
     T = w.n_tokens
     attn_bytes = kv_rows * Hkv * d * 2 * 2 + T * Hq * d * 2 * 2
     append_bytes = T * Hkv * d * 2 * 2 * 2 + T * Hq * d * 2 * 2
-    flops = 4 * d * Hq * pairs
-    return {"attn_bytes": attn_bytes, "append_bytes": append_bytes, "flops": flops,
-            "pairs": pairs, "kv_rows": kv_rows}
+    return {"attn_bytes": attn_bytes, "append_bytes": append_bytes, "flops": 4 * d * Hq * pairs,
+            "pairs": pairs, "kv_rows": kv_rows,
+            "decode_bytes": dec_rows * Hkv * d * 2 * 2 + dec_tokens * Hq * d * 2 * 2,
+            "tc_flops": 4 * d * Hq * tc_pairs,
+            "tc_bytes": tc_rows * Hkv * d * 2 * 2 + (T - dec_tokens) * Hq * d * 2 * 2}
+
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch, from one ncu capture
+# of the kernel on the headline batch (compact pool); None once the kernel has
+# changed since that capture. Summaries with the commands are in profiles/.
+NCU_TRAFFIC = {
+    "decode": 1.260098e9 + 6.556672e6,
+    "tc": None,
+}
 
 
 def load_peaks():
@@ -285,6 +306,19 @@ def run_fg(args, w, rank, ws, local_rank):
     batch.device_status(stream)
     info = batch.plan_info()
 
+    # per-kernel durations: the library's own CUDA events around each kernel,
+    # on the stream it runs on (a separate pass, synchronised per step so
+    # the events of every step can be read; the kernels run exactly as above)
+    batch.set_timing(True)
+    kms = []
+    for _ in range(args.steps):
+        step(mk())
+        kms.append(batch.kernel_ms())
+        flush_l2()
+    batch.set_timing(False)
+    torch.cuda.synchronize()
+    kernel_ms = {k: max_over_ranks(sum(d[k] for d in kms) / len(kms), dev) for k in kms[0]}
+
     # end to end through the public API from pinned host buffers
     host_in = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v))}
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -318,8 +352,27 @@ def run_fg(args, w, rank, ws, local_rank):
         return 0
     work = algorithmic_work(w)
     hbm, tf, src = load_peaks()
-    achieved = work["attn_bytes"] / (attn_ms_mean / 1000) / 1e9
     tokens = w.n_tokens * ws
+    # roofline of the dominant kernel (longest average launch)
+    dom = max(("decode", "tc"), key=lambda k: kernel_ms[k])
+    if dom == "decode":
+        achieved = work["decode_bytes"] / (kernel_ms["decode"] / 1000) / 1e9
+        roof = {"kernel": "attn_decode_kernel (MHA split-KV decode)", "bound": "hbm",
+                "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": NCU_TRAFFIC["decode"], "algorithmic_bytes": work["decode_bytes"]}
+    else:
+        achieved = work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12
+        roof = {"kernel": "attn_tc_kernel (tcgen05 tiles)", "bound": "tensor", "achieved": achieved,
+                "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf, "traffic": NCU_TRAFFIC["tc"],
+                "algorithmic_flops": work["tc_flops"]}
+    roof.update({"peak_source": f"{src} (MEASURED_PEAKS.json)" if src == "measured" else src,
+                 "kernel_ms": kernel_ms,
+                 "attention_call_ms": attn_ms_mean,
+                 "attention_call_GBps": work["attn_bytes"] / (attn_ms_mean / 1000) / 1e9,
+                 "tc_TFLOPs": work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12 if kernel_ms["tc"] else None,
+                 "step_roofline_ms": 1000 * max((work["attn_bytes"] + work["append_bytes"]) / (hbm * 1e9),
+                                                work["flops"] / (tf * 1e12))})
+    roof["step_frac"] = roof["step_roofline_ms"] / ms
     line = {
         "metric": METRIC, "value": tokens / (ms / 1000), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -329,14 +382,7 @@ def run_fg(args, w, rank, ws, local_rank):
                    "head_dim": w.head_dim, "block_size": w.block_size, "pool_blocks": w.n_blocks,
                    "note": w.note, "l2": "flushed between steps (256 MB write, outside the events)",
                    "parallelism": f"replicas x{ws}"},
-        "roofline": {"kernel": "ragged attention (work units + split-KV combine)", "bound": "hbm",
-                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": None, "peak_source": src,
-                     "attn_ms": attn_ms_mean, "algorithmic_bytes": work["attn_bytes"],
-                     "flops": work["flops"],
-                     "tflops_achieved": work["flops"] / (attn_ms_mean / 1000) / 1e12,
-                     "step_roofline_ms": 1000 * max((work["attn_bytes"] + work["append_bytes"]) / (hbm * 1e9),
-                                                    work["flops"] / (tf * 1e12))},
+        "roofline": roof,
         "e2e": {"value": tokens / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * (1 + info["launches"]),

@@ -198,6 +198,16 @@ fg_status fg_ragged_attention_noalloc(const fg_kv_cache* cache, fg_ragged_batch*
  * info[6..7] = 0. */
 fg_status fg_attention_plan_info(const fg_ragged_batch* batch, int32_t info[8]);
 
+/* Kernel timing for profiling. With `enable` != 0, each later
+ * fg_ragged_attention call on this batch records CUDA events around its
+ * kernels, on the streams they run on; fg_attention_kernel_ms then waits for
+ * the last call's events and returns the duration in milliseconds of
+ * ms[0] = MHA split-KV decode kernel, ms[1] = tensor-core kernel,
+ * ms[2] = general-path kernel, ms[3] = combine kernel (0 where a kernel did
+ * not run). Off by default. */
+fg_status fg_ragged_batch_set_timing(fg_ragged_batch* batch, int32_t enable);
+fg_status fg_attention_kernel_ms(fg_ragged_batch* batch, float ms[4]);
+
 /* Reads (and clears) the batch's device error word after synchronising
  * `stream`: FG_OK, or FG_ERR_DEVICE_CHECK if a kernel met an index outside
  * its buffers (the access was skipped), or FG_ERR_TIMEOUT. */

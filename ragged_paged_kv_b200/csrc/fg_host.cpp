@@ -144,6 +144,13 @@ struct fg_ragged_batch {
   size_t dplan_bytes = 0;
   Staging plan_stage;
   int32_t last_launches = 0;
+  // second stream: tensor-core tiles run beside the decode kernel
+  cudaStream_t aux = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  // optional kernel timing: begin/end events of decode, tc, general, combine
+  bool timing = false;
+  cudaEvent_t tev[8] = {};
+  bool tran[4] = {};
   // split-KV partials
   float* ws = nullptr;
   size_t ws_bytes = 0;
@@ -314,6 +321,11 @@ extern "C" fg_status fg_ragged_batch_destroy(fg_ragged_batch* b) {
   if (b->derr) cudaFree(b->derr);
   if (b->dplan) cudaFree(b->dplan);
   if (b->ws) cudaFree(b->ws);
+  for (cudaEvent_t e : b->tev)
+    if (e) cudaEventDestroy(e);
+  if (b->aux) cudaStreamDestroy(b->aux);
+  if (b->fork) cudaEventDestroy(b->fork);
+  if (b->join) cudaEventDestroy(b->join);
   delete b;
   return FG_OK;
 }
@@ -578,6 +590,30 @@ bool make_q_map(CUtensorMap* m, const void* q_rot, int T, int Hq, int d, int g) 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int sm_count() {
+  static int n[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!n[dev] && cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    n[dev] = 148;
+  return n[dev];
+}
+
+// Persistent grid of the tensor-core kernel: two CTAs per SM when it runs
+// alone; one when the decode kernel shares the SMs (a decode CTA then fits
+// beside each tensor-core CTA).
+int tc_grid(const fg::Plan& P) { return sm_count() * (P.n_decode > 0 ? 1 : 2); }
+
+fg_status ensure_aux_stream(fg_ragged_batch* b) {
+  if (b->aux) return FG_OK;
+  int lo = 0, hi = 0;
+  FG_CUDA(cudaDeviceGetStreamPriorityRange(&lo, &hi));
+  FG_CUDA(cudaStreamCreateWithPriority(&b->aux, cudaStreamNonBlocking, hi));
+  FG_CUDA(cudaEventCreateWithFlags(&b->fork, cudaEventDisableTiming));
+  FG_CUDA(cudaEventCreateWithFlags(&b->join, cudaEventDisableTiming));
+  return FG_OK;
+}
+
 bool tc_eligible(fg_kv_cache* c, int g) {
   const bool pow2 = g >= 1 && g <= fg::kTcRows && (g & (g - 1)) == 0;
   return pow2 && ensure_kv_map(c);
@@ -678,24 +714,77 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   const CacheView cv = cache_view(c);
   const auto* qr = static_cast<const __nv_bfloat16*>(q_rot);
   auto* o = static_cast<__nv_bfloat16*>(out);
+  // optional timing events around each kernel, on its own stream
+  auto mark = [&](int k, int end, cudaStream_t st_) -> fg_status {
+    if (!b->timing) return FG_OK;
+    FG_CUDA(cudaEventRecord(b->tev[2 * k + end], st_));
+    b->tran[k] = true;
+    return FG_OK;
+  };
+  if (b->timing)
+    for (bool& r : b->tran) r = false;
+  if (P.n_general && (st = mark(2, 0, strm))) return st;
   cudaError_t e = fg::launch_attention_general(
       cv, b->view, reinterpret_cast<const WorkItem*>(base + P.off_general), P.n_general, qr, o,
       part_o, part_ml, n_q_heads, g, scale_log2, window, strm);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  if (P.n_general && (st = mark(2, 1, strm))) return st;
+  // tensor-core tiles and MHA decode units touch disjoint outputs and
+  // partial rows: run them side by side (tc on a high-priority second
+  // stream forked from and joined back into the caller's stream)
+  const bool both = P.n_tc > 0 && P.n_decode > 0;
+  cudaStream_t tc_stream = strm;
+  if (both) {
+    st = ensure_aux_stream(b);
+    if (st) return st;
+    FG_CUDA(cudaEventRecord(b->fork, strm));
+    FG_CUDA(cudaStreamWaitEvent(b->aux, b->fork, 0));
+    tc_stream = b->aux;
+  }
+  if (P.n_tc) {
+    if ((st = mark(1, 0, tc_stream))) return st;
+    e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
+                                reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
+                                part_ml, n_q_heads, g, scale_log2, window, tc_grid(P), tc_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
+    if ((st = mark(1, 1, tc_stream))) return st;
+  }
+  if (P.n_decode && (st = mark(0, 0, strm))) return st;
   e = fg::launch_attention_decode(cv, b->view,
                                   reinterpret_cast<const WorkItem*>(base + P.off_decode), P.n_decode,
                                   qr, o, part_o, part_ml, n_q_heads, scale_log2, strm);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
-  if (P.n_tc) {
-    e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
-                                reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
-                                part_ml, n_q_heads, g, scale_log2, window, strm);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
+  if (P.n_decode && (st = mark(0, 1, strm))) return st;
+  if (both) {
+    FG_CUDA(cudaEventRecord(b->join, b->aux));
+    FG_CUDA(cudaStreamWaitEvent(strm, b->join, 0));
   }
+  if (P.n_combine && (st = mark(3, 0, strm))) return st;
   e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),
                          P.n_combine, P.max_combine_rows, part_o, part_ml, o, n_q_heads, g,
                          c->head_dim, strm);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  if (P.n_combine && (st = mark(3, 1, strm))) return st;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_ragged_batch_set_timing(fg_ragged_batch* b, int32_t enable) {
+  if (!b) return fail(FG_ERR_INVALID_ARG, "batch is NULL");
+  if (enable)
+    for (cudaEvent_t& e : b->tev)
+      if (!e) FG_CUDA(cudaEventCreate(&e));
+  b->timing = enable != 0;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_attention_kernel_ms(fg_ragged_batch* b, float ms[4]) {
+  if (!b || !ms) return fail(FG_ERR_INVALID_ARG, "NULL argument");
+  for (int k = 0; k < 4; ++k) {
+    ms[k] = 0.f;
+    if (!b->timing || !b->tran[k]) continue;
+    FG_CUDA(cudaEventSynchronize(b->tev[2 * k + 1]));
+    FG_CUDA(cudaEventElapsedTime(&ms[k], b->tev[2 * k], b->tev[2 * k + 1]));
+  }
   return FG_OK;
 }
 
@@ -799,7 +888,7 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
   if (P.n_tc) {
     e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
-                                part_ml, n_q_heads, g, scale_log2, window, strm);
+                                part_ml, n_q_heads, g, scale_log2, window, 2 * sm_count(), strm);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
   }
   e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),

@@ -86,7 +86,7 @@ cudaError_t launch_attention_decode(const CacheView& cache, const BatchView& bat
 cudaError_t launch_attention_tc(const void* tm_q, const void* tm_kv, const CacheView& cache,
                                 const BatchView& batch, const WorkItem* items, int n_items,
                                 __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
-                                int g, float scale_log2, int window, cudaStream_t stream);
+                                int g, float scale_log2, int window, int grid, cudaStream_t stream);
 
 cudaError_t launch_combine(const BatchView& batch, const CombineItem* items, int n_items,
                            int max_rows, const float* part_o, const float* part_ml,

@@ -53,6 +53,8 @@ def lib() -> ctypes.CDLL:
         "fg_ragged_attention_noalloc": [V, V, V, V, I32, F, I32, V],
         "fg_device_status": [V, V],
         "fg_attention_plan_info": [V, _c_int32_p],
+        "fg_ragged_batch_set_timing": [V, I32],
+        "fg_attention_kernel_ms": [V, _c_float_p],
         "fg_rotary_table": [D, I32, I32, I32, _c_float_p, _c_float_p],
     }
     for name, args in sig.items():
@@ -200,6 +202,15 @@ class RaggedBatch:
         keys = ("general_units", "decode_units", "tensor_units", "combine_groups", "partial_rows",
                 "launches")
         return dict(zip(keys, list(a)[:6]))
+
+    def set_timing(self, enable: bool = True):
+        _check(lib().fg_ragged_batch_set_timing(self._h, 1 if enable else 0), "fg_ragged_batch_set_timing")
+
+    def kernel_ms(self) -> dict:
+        """Durations (ms) of the last attention call's kernels (timing must be on)."""
+        a = (ctypes.c_float * 4)()
+        _check(lib().fg_attention_kernel_ms(self._h, ctypes.cast(a, _c_float_p)), "fg_attention_kernel_ms")
+        return dict(zip(("decode", "tc", "general", "combine"), list(a)))
 
     def device_status(self, stream=None):
         _check(lib().fg_device_status(self._h, _stream_ptr(stream)), "fg_device_status")
