@@ -84,7 +84,7 @@ def algorithmic_work(w):
     Hq, Hkv, d, W = w.n_q_heads, w.n_kv_heads, w.head_dim, w.sliding_window
     g = Hq // Hkv
     kv_rows = pairs = 0
-    dec_rows = dec_tokens = 0      # one-token MHA decodes: the split-KV decode kernel
+    dec_rows = dec_tokens = 0      # one-token decodes: the decode kernels
     tc_pairs = tc_rows = 0         # everything else: the tensor-core kernel
     for q, c in zip(w.q_lens.tolist(), w.ctx_lens.tolist()):
         p = np.arange(c, c + q, dtype=np.int64)
@@ -93,7 +93,7 @@ def algorithmic_work(w):
         prs = int((p - lo + 1).sum())
         kv_rows += rows
         pairs += prs
-        if q == 1 and g == 1:
+        if q == 1 and (g == 1 or (d == 128 and g <= 16)):   # the decode kernels
             dec_rows += rows
             dec_tokens += 1
         else:
@@ -105,6 +105,7 @@ def algorithmic_work(w):
     return {"attn_bytes": attn_bytes, "append_bytes": append_bytes, "flops": 4 * d * Hq * pairs,
             "pairs": pairs, "kv_rows": kv_rows,
             "decode_bytes": dec_rows * Hkv * d * 2 * 2 + dec_tokens * Hq * d * 2 * 2,
+            "decode_flops": 4 * d * Hq * (pairs - tc_pairs),
             "tc_flops": 4 * d * Hq * tc_pairs,
             "tc_bytes": tc_rows * Hkv * d * 2 * 2 + (T - dec_tokens) * Hq * d * 2 * 2}
 
@@ -113,7 +114,7 @@ def algorithmic_work(w):
 # of the kernel on the headline batch (compact pool); None once the kernel has
 # changed since that capture. Summaries with the commands are in profiles/.
 NCU_TRAFFIC = {
-    "decode": 1.260098e9 + 6.556672e6,
+    "decode": None,
     "tc": None,
 }
 
@@ -262,8 +263,11 @@ def run_fg(args, w, rank, ws, local_rank):
     stream = torch.cuda.Stream(device=dev)
     cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim, device=dev)
     fixtures.fill(cache.tensor, 0)
-    fixtures.write_context(w, cache.tensor)
+    # prior context: seeded N(0,1) bf16 blocks (a pool of them, reused across
+    # sequences: same sizes and distribution, fast to set up for any pool)
+    fixtures.write_context(w, cache.tensor, keep=(), others="pool")
     batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+    batch.set_overlap(args.overlap)
     q, k, v = fixtures.qkv_device(w, dev)
     q_rot, out = torch.empty_like(q), torch.empty_like(q)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -292,13 +296,17 @@ def run_fg(args, w, rank, ws, local_rank):
     evs = [mk() for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
+    host_s = 0.0
     with ClockSampler(local_rank) as clocks:
         for i in range(args.steps):
+            t0 = time.perf_counter()
             step(evs[i])
+            host_s += time.perf_counter() - t0
             flush_l2()
         torch.cuda.synchronize()
     barrier()
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    put_append_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / len(evs)
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
     ms_local = sum(step_ms) / len(step_ms)
     ms = max_over_ranks(ms_local, dev)
@@ -357,17 +365,24 @@ def run_fg(args, w, rank, ws, local_rank):
     dom = max(("decode", "tc"), key=lambda k: kernel_ms[k])
     if dom == "decode":
         achieved = work["decode_bytes"] / (kernel_ms["decode"] / 1000) / 1e9
-        roof = {"kernel": "attn_decode_kernel (MHA split-KV decode)", "bound": "hbm",
+        roof = {"kernel": "decode (attn_decode_tc_kernel at d=128, attn_decode_kernel at d=64)", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": NCU_TRAFFIC["decode"], "algorithmic_bytes": work["decode_bytes"]}
-    else:
+    elif work["tc_flops"] / (tf * 1e12) >= work["tc_bytes"] / (hbm * 1e9):
         achieved = work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12
         roof = {"kernel": "attn_tc_kernel (tcgen05 tiles)", "bound": "tensor", "achieved": achieved,
                 "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf, "traffic": NCU_TRAFFIC["tc"],
                 "algorithmic_flops": work["tc_flops"]}
+    else:  # its tiles are mostly grouped-query decodes: bound by the K/V bytes
+        achieved = work["tc_bytes"] / (kernel_ms["tc"] / 1000) / 1e9
+        roof = {"kernel": "attn_tc_kernel (tcgen05 tiles)", "bound": "hbm", "achieved": achieved,
+                "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": NCU_TRAFFIC["tc"],
+                "algorithmic_bytes": work["tc_bytes"]}
     roof.update({"peak_source": f"{src} (MEASURED_PEAKS.json)" if src == "measured" else src,
                  "kernel_ms": kernel_ms,
                  "attention_call_ms": attn_ms_mean,
+                 "put_append_ms": put_append_ms,
+                 "host_enqueue_ms_per_step": 1000 * host_s / args.steps,
                  "attention_call_GBps": work["attn_bytes"] / (attn_ms_mean / 1000) / 1e9,
                  "tc_TFLOPs": work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12 if kernel_ms["tc"] else None,
                  "step_roofline_ms": 1000 * max((work["attn_bytes"] + work["append_bytes"]) / (hbm * 1e9),
@@ -377,7 +392,7 @@ def run_fg(args, w, rank, ws, local_rank):
         "metric": METRIC, "value": tokens / (ms / 1000), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{w.name} (Llama-2-7B attention shape)", "tokens_per_gpu": w.n_tokens,
+        "config": {"workload": f"{w.name} ({w.n_q_heads}/{w.n_kv_heads} heads, d={w.head_dim})", "tokens_per_gpu": w.n_tokens,
                    "seqs": w.n_seqs, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
                    "head_dim": w.head_dim, "block_size": w.block_size, "pool_blocks": w.n_blocks,
                    "note": w.note, "l2": "flushed between steps (256 MB write, outside the events)",
@@ -386,7 +401,7 @@ def run_fg(args, w, rank, ws, local_rank):
         "e2e": {"value": tokens / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * (1 + info["launches"]),
-        "plan": info,
+        "plan": dict(info, overlap=args.overlap),
         "clocks": clocks.summary(),
     }
     if ws == 1 and not args.no_cpu_baseline:
@@ -403,13 +418,20 @@ def main():
     ap.add_argument("--impl", choices=["fg", "reference"], default="fg")
     ap.add_argument("--config", type=int, default=2, help="workload number (2 = the headline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--overlap", action="store_true",
+                    help="run the query-tile kernel beside the decode kernel on a second stream")
     ap.add_argument("--compact-pool", action="store_true",
                     help="size the block pool to what the batch uses (small ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from ragged_paged_kv_b200 import workloads as W
-    w = W.CONFIGS[args.config]()
+    if args.config == 3 and args.impl == "fg":
+        import torch
+        free, _ = torch.cuda.mem_get_info(world()[2])
+        w = W.config3(n_blocks=int(min(180 * 10**9, free - 8 * 2**30) // (2 * 32 * 64 * 128 * 2)))
+    else:
+        w = W.CONFIGS[args.config]()
     if args.compact_pool:
         need = sum(w.blocks_used(s) for s in range(w.n_seqs))
         w = W._make(w.name, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.seq_ids,

@@ -208,6 +208,16 @@ fg_status fg_attention_plan_info(const fg_ragged_batch* batch, int32_t info[8]);
 fg_status fg_ragged_batch_set_timing(fg_ragged_batch* batch, int32_t enable);
 fg_status fg_attention_kernel_ms(fg_ragged_batch* batch, float ms[4]);
 
+/* Scheduling of one attention call that has both one-token decode units and
+ * prompt-chunk query tiles. enable == 0 (default): the two kernels run one
+ * after the other on the caller's stream, each with the whole GPU (two CTAs
+ * per SM). enable != 0: the query-tile kernel runs on a second,
+ * high-priority stream beside the decode kernel, each sized for one CTA per
+ * SM. On a B200 the default is faster (the hardware may place two CTAs of
+ * one kernel on an SM, which unbalances the persistent grids). Results are
+ * identical either way. */
+fg_status fg_ragged_batch_set_overlap(fg_ragged_batch* batch, int32_t enable);
+
 /* Reads (and clears) the batch's device error word after synchronising
  * `stream`: FG_OK, or FG_ERR_DEVICE_CHECK if a kernel met an index outside
  * its buffers (the access was skipped), or FG_ERR_TIMEOUT. */

@@ -148,6 +148,7 @@ struct fg_ragged_batch {
   cudaStream_t aux = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
   // optional kernel timing: begin/end events of decode, tc, general, combine
+  bool overlap = false;
   bool timing = false;
   cudaEvent_t tev[8] = {};
   bool tran[4] = {};
@@ -578,12 +579,15 @@ bool ensure_kv_map(fg_kv_cache* c) {
 // q_rot as a 3-D bf16 tensor (head_dim, n_q_heads, tokens); a box of
 // 64 dims x g heads x 128/g tokens lands as 128 rows (token-major, head-minor)
 // of 128 bytes, the A-operand layout of a query tile.
-bool make_q_map(CUtensorMap* m, const void* q_rot, int T, int Hq, int d, int g) {
+// tokens_per_box = 1 gives the decode kernel's view: g rows of one token.
+bool make_q_map(CUtensorMap* m, const void* q_rot, int T, int Hq, int d, int g,
+                int tokens_per_box = 0) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)Hq, (cuuint64_t)T};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)Hq * d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)g, (cuuint32_t)(fg::kTcRows / g)};
+  cuuint32_t box[3] = {64, (cuuint32_t)g,
+                       (cuuint32_t)(tokens_per_box > 0 ? tokens_per_box : fg::kTcRows / g)};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q_rot), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -599,10 +603,13 @@ int sm_count() {
   return n[dev];
 }
 
-// Persistent grid of the tensor-core kernel: two CTAs per SM when it runs
-// alone; one when the decode kernel shares the SMs (a decode CTA then fits
-// beside each tensor-core CTA).
-int tc_grid(const fg::Plan& P) { return sm_count() * (P.n_decode > 0 ? 1 : 2); }
+// Persistent grids: two CTAs per SM for a kernel that runs alone; one each
+// when the query-tile kernel and a decode kernel share the SMs (a decode CTA
+// then fits beside each query-tile CTA).
+bool overlapped(const fg::Plan& P, bool overlap) {
+  return overlap && P.n_tc > 0 && (P.n_decode > 0 || P.n_dtc > 0);
+}
+int tc_grid(const fg::Plan& P, bool overlap) { return sm_count() * (overlapped(P, overlap) ? 1 : 2); }
 
 fg_status ensure_aux_stream(fg_ragged_batch* b) {
   if (b->aux) return FG_OK;
@@ -692,8 +699,9 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   const bool use_tc = tc_eligible(const_cast<fg_kv_cache*>(c), g);
   if (!use_tc && g > fg::kMaxGroup)
     return fail(FG_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads = %d > %d", g, fg::kMaxGroup);
-  CUtensorMap tm_q;
-  if (use_tc && !make_q_map(&tm_q, q_rot, b->n_tokens, n_q_heads, c->head_dim, g))
+  CUtensorMap tm_q, tm_q1;
+  if (use_tc && (!make_q_map(&tm_q, q_rot, b->n_tokens, n_q_heads, c->head_dim, g) ||
+                 !make_q_map(&tm_q1, q_rot, b->n_tokens, n_q_heads, c->head_dim, g, 1)))
     return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q_rot");
   st = prepare_plan(b, c, g, window, use_tc, strm);
   if (st) return st;
@@ -709,7 +717,8 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   float* part_o = ws;
   float* part_ml = ws ? ws + (size_t)P.part_rows * c->head_dim : nullptr;
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
-  b->last_launches = (P.n_general > 0) + (P.n_decode > 0) + (P.n_tc > 0) + (P.n_combine > 0);
+  b->last_launches = (P.n_general > 0) + (P.n_decode > 0) + (P.n_tc > 0) + (P.n_dtc > 0) +
+                     (P.n_combine > 0);
   const char* base = static_cast<const char*>(b->dplan);
   const CacheView cv = cache_view(c);
   const auto* qr = static_cast<const __nv_bfloat16*>(q_rot);
@@ -732,7 +741,7 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   // tensor-core tiles and MHA decode units touch disjoint outputs and
   // partial rows: run them side by side (tc on a high-priority second
   // stream forked from and joined back into the caller's stream)
-  const bool both = P.n_tc > 0 && P.n_decode > 0;
+  const bool both = overlapped(P, b->overlap);
   cudaStream_t tc_stream = strm;
   if (both) {
     st = ensure_aux_stream(b);
@@ -745,7 +754,8 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
     if ((st = mark(1, 0, tc_stream))) return st;
     e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
-                                part_ml, n_q_heads, g, scale_log2, window, tc_grid(P), tc_stream);
+                                part_ml, n_q_heads, g, scale_log2, window, tc_grid(P, b->overlap),
+                                tc_stream);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
     if ((st = mark(1, 1, tc_stream))) return st;
   }
@@ -755,6 +765,15 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
                                   qr, o, part_o, part_ml, n_q_heads, scale_log2, strm);
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
   if (P.n_decode && (st = mark(0, 1, strm))) return st;
+  if (P.n_dtc) {
+    if ((st = mark(0, 0, strm))) return st;
+    e = fg::launch_attention_decode_tc(&tm_q1, &c->tm_kv, cv, b->view,
+                                       reinterpret_cast<const WorkItem*>(base + P.off_dtc), P.n_dtc, o,
+                                       part_o, part_ml, n_q_heads, g, scale_log2,
+                                       sm_count() * (both ? 1 : 2), strm);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core decode launch");
+    if ((st = mark(0, 1, strm))) return st;
+  }
   if (both) {
     FG_CUDA(cudaEventRecord(b->join, b->aux));
     FG_CUDA(cudaStreamWaitEvent(strm, b->join, 0));
@@ -765,6 +784,12 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
                          c->head_dim, strm);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   if (P.n_combine && (st = mark(3, 1, strm))) return st;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_ragged_batch_set_overlap(fg_ragged_batch* b, int32_t enable) {
+  if (!b) return fail(FG_ERR_INVALID_ARG, "batch is NULL");
+  b->overlap = enable != 0;
   return FG_OK;
 }
 
@@ -792,7 +817,7 @@ extern "C" fg_status fg_attention_plan_info(const fg_ragged_batch* b, int32_t in
   if (!b || !info) return fail(FG_ERR_INVALID_ARG, "NULL argument");
   const fg::Plan& P = b->plan;
   info[0] = P.n_general;
-  info[1] = P.n_decode;
+  info[1] = P.n_decode + P.n_dtc;
   info[2] = P.n_tc;
   info[3] = P.n_combine;
   info[4] = P.part_rows;
@@ -854,8 +879,9 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
   const bool use_tc = tc_eligible(const_cast<fg_kv_cache*>(c), g);
   if (!use_tc && g > fg::kMaxGroup)
     return fail(FG_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads = %d > %d", g, fg::kMaxGroup);
-  CUtensorMap tm_q;
-  if (use_tc && !make_q_map(&tm_q, q_rot, b->n_tokens, n_q_heads, c->head_dim, g))
+  CUtensorMap tm_q, tm_q1;
+  if (use_tc && (!make_q_map(&tm_q, q_rot, b->n_tokens, n_q_heads, c->head_dim, g) ||
+                 !make_q_map(&tm_q1, q_rot, b->n_tokens, n_q_heads, c->head_dim, g, 1)))
     return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q_rot");
   thread_local fg::Plan P;
   thread_local std::vector<unsigned char> packed;
@@ -890,6 +916,12 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
                                 part_ml, n_q_heads, g, scale_log2, window, 2 * sm_count(), strm);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
+  }
+  if (P.n_dtc) {
+    e = fg::launch_attention_decode_tc(&tm_q1, &c->tm_kv, cv, b->view,
+                                       reinterpret_cast<const WorkItem*>(base + P.off_dtc), P.n_dtc, o,
+                                       part_o, part_ml, n_q_heads, g, scale_log2, 2 * sm_count(), strm);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core decode launch");
   }
   e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),
                          P.n_combine, P.max_combine_rows, part_o, part_ml, o, n_q_heads, g,

@@ -12,6 +12,7 @@ void Plan::pack(void* dst) const {
   if (n_general) std::memcpy(p + off_general, general.data(), general.size() * sizeof(WorkItem));
   if (n_decode) std::memcpy(p + off_decode, decode.data(), decode.size() * sizeof(WorkItem));
   if (n_tc) std::memcpy(p + off_tc, tc.data(), tc.size() * sizeof(WorkItem));
+  if (n_dtc) std::memcpy(p + off_dtc, dtc.data(), dtc.size() * sizeof(WorkItem));
   if (n_combine) std::memcpy(p + off_combine, combine.data(), combine.size() * sizeof(CombineItem));
 }
 
@@ -22,6 +23,7 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
   P.general.clear();
   P.decode.clear();
   P.tc.clear();
+  P.dtc.clear();
   P.combine.clear();
   P.part_rows = 0;
   P.max_combine_rows = 0;
@@ -50,6 +52,11 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
   };
   for (int s = 0; s < S; ++s) {
     const int q = q_lens[s], c = ctx_lens[s];
+    if (use_tc && q == 1 && head_dim == 128 && g <= kDtcMaxGroup) {
+      const int kb = window > 0 ? std::max(0, c - window + 1) : 0;
+      for (int h = 0; h < n_kv_heads; ++h) emit(P.dtc, s, h, 0, 1, kb, c + 1, kTcDecodeSplitKeys);
+      continue;
+    }
     if (q == 1 && g == 1) {
       const int kb = window > 0 ? std::max(0, c - window + 1) : 0;
       for (int h = 0; h < n_kv_heads; ++h) emit(P.decode, s, h, 0, 1, kb, c + 1, kDecodeSplitKeys);
@@ -77,17 +84,21 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
   std::stable_sort(P.decode.begin(), P.decode.end(), [](const WorkItem& a, const WorkItem& b) {
     return a.key_end - a.key_begin > b.key_end - b.key_begin;
   });
-  std::stable_sort(P.tc.begin(), P.tc.end(), [](const WorkItem& a, const WorkItem& b) {
+  auto longest_first = [](const WorkItem& a, const WorkItem& b) {
     return a.key_end - a.key_begin > b.key_end - b.key_begin;
-  });
+  };
+  std::stable_sort(P.tc.begin(), P.tc.end(), longest_first);
+  std::stable_sort(P.dtc.begin(), P.dtc.end(), longest_first);
   P.n_general = (int32_t)P.general.size();
   P.n_decode = (int32_t)P.decode.size();
   P.n_tc = (int32_t)P.tc.size();
+  P.n_dtc = (int32_t)P.dtc.size();
   P.n_combine = (int32_t)P.combine.size();
   P.off_general = 0;
   P.off_decode = align_up(P.general.size() * sizeof(WorkItem), 256);
   P.off_tc = align_up(P.off_decode + P.decode.size() * sizeof(WorkItem), 256);
-  P.off_combine = align_up(P.off_tc + P.tc.size() * sizeof(WorkItem), 256);
+  P.off_dtc = align_up(P.off_tc + P.tc.size() * sizeof(WorkItem), 256);
+  P.off_combine = align_up(P.off_dtc + P.dtc.size() * sizeof(WorkItem), 256);
   P.total = align_up(P.off_combine + P.combine.size() * sizeof(CombineItem), 256);
 }
 

@@ -15,17 +15,19 @@ constexpr int kSplitKeys = 1024;  // keys per split-KV partial (general path)
 constexpr int kDecodeSplitKeys = 512;  // keys per unit of the MHA decode kernel
 constexpr int kTcRows = 128;           // query rows per tensor-core tile
 constexpr int kTcDecodeSplitKeys = 2048;  // keys per unit for small (decode) tc tiles
+constexpr int kDtcMaxGroup = 16;          // q heads per kv head the decode tc kernel serves
 
 struct Plan {
   std::vector<WorkItem> general;   // CUDA-core general path
   std::vector<WorkItem> decode;    // one-row MHA decode units (split-KV)
-  std::vector<WorkItem> tc;        // tensor-core tiles (prefill chunks, grouped decode)
+  std::vector<WorkItem> tc;        // tensor-core query tiles (prompt chunks)
+  std::vector<WorkItem> dtc;       // one-token decodes on tensor cores (keys as MMA rows)
   std::vector<CombineItem> combine;
   int32_t part_rows = 0;         // partial rows the split units write
   int32_t max_combine_rows = 0;  // largest n_rows among combine items
   // packed device layout (bytes from the plan buffer's start)
-  size_t off_general = 0, off_decode = 0, off_tc = 0, off_combine = 0, total = 0;
-  int32_t n_general = 0, n_decode = 0, n_tc = 0, n_combine = 0;
+  size_t off_general = 0, off_decode = 0, off_tc = 0, off_dtc = 0, off_combine = 0, total = 0;
+  int32_t n_general = 0, n_decode = 0, n_tc = 0, n_dtc = 0, n_combine = 0;
 
   size_t bytes() const { return total; }
   void pack(void* dst) const;
@@ -37,8 +39,11 @@ struct Plan {
 // kernel. One-token queries with one q head per kv head go to the decode
 // kernel in kDecodeSplitKeys-key units; everything else to the general path
 // (up to kGeneralRows rows per unit, kSplitKeys keys per partial).
-// use_tc: the tensor-core kernel may serve every unit that is not an MHA
-// decode (requires g a power of two <= 128).
+// use_tc: the tensor-core kernels may serve the batch (tensor maps built,
+// g a power of two <= 128). Then one-token decodes with d = 128 and g <= 16
+// go to the keys-as-rows decode kernel (dtc), other tokens to 128-row query
+// tiles (tc); without it, MHA decodes go to the CUDA-core decode kernel and
+// the rest to the general path.
 void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& ctx_lens,
                 int n_kv_heads, int g, int head_dim, int window, bool use_tc, Plan* out);
 

@@ -4,7 +4,8 @@
 //
 // One CTA per batch row (token). Each thread rotates 8 (i, i + d/2) pairs at a
 // time with 16-byte loads of both halves and writes 16-byte stores, so every
-// global access is a full, aligned 16-byte vector. The rotation runs in double
+// global access is a full, aligned 16-byte vector; a thread issues the loads
+// of four heads before it computes and stores any of them. The rotation runs in double
 // so that it rounds exactly once: a bf16 times a float product is exact in
 // double (8 + 24 significant bits), the sum rounds once, and the double is
 // rounded straight to bf16 (ties to even) - no float intermediate that could
@@ -28,6 +29,10 @@ __device__ __forceinline__ unsigned short f64_to_bf16_rne(double x) {
 __device__ __forceinline__ double bf16_lo(uint32_t w) { return (double)__uint_as_float(w << 16); }
 __device__ __forceinline__ double bf16_hi(uint32_t w) { return (double)__uint_as_float(w & 0xFFFF0000u); }
 
+__device__ __forceinline__ const __nv_bfloat16* k_in(const __nv_bfloat16* k, int t, int Hkv, int h, int D) {
+  return k + ((int64_t)t * Hkv + h) * D;
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) rotary_append_kernel(CacheView cache, BatchView batch,
                                                             const __nv_bfloat16* q,
@@ -47,56 +52,84 @@ __global__ void __launch_bounds__(128) rotary_append_kernel(CacheView cache, Bat
   int32_t blk = batch.bt[batch.bt_off[s] + lb];
   const bool blk_ok = blk >= 0 && blk < cache.n_blocks;
   if (!blk_ok && threadIdx.x == 0) atomicOr(batch.err, kErrBadBlock);
-
-  const float2* rp = rope + (int64_t)p * HALF;
-  const int total = (Hq + Hkv) * GROUPS;
-  for (int gi = threadIdx.x; gi < total; gi += blockDim.x) {
-    const int h = gi / GROUPS;
-    const int i0 = (gi - h * GROUPS) * 8;
-    const bool is_q = h < Hq;
-    const __nv_bfloat16* src = is_q ? q + ((int64_t)t * Hq + h) * D
-                                    : k + ((int64_t)t * Hkv + (h - Hq)) * D;
-    const uint4 a = *reinterpret_cast<const uint4*>(src + i0);
-    const uint4 b = *reinterpret_cast<const uint4*>(src + HALF + i0);
-    const float4* r4 = reinterpret_cast<const float4*>(rp + i0);
-    float cs[8], sn[8];
+  // Every thread handles the same 8-pair group i0 of several heads (the block
+  // size is a multiple of the groups per head), so its 8 (cos, sin) pairs are
+  // loaded once; all loads of a batch of heads are issued before any store.
+  static_assert(128 % GROUPS == 0, "block size must be a multiple of the groups per head");
+  const int i0 = (threadIdx.x % GROUPS) * 8;
+  float cs[8], sn[8];
+  {
+    const float4* r4 = reinterpret_cast<const float4*>(rope + (int64_t)p * HALF + i0);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float4 r = r4[e];
       cs[2 * e] = r.x; sn[2 * e] = r.y; cs[2 * e + 1] = r.z; sn[2 * e + 1] = r.w;
     }
-    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-    uint32_t y1[4], y2[4];
+  }
+  constexpr int BATCH = 4;
+  const int total = (Hq + Hkv) * GROUPS;
+  for (int base = threadIdx.x; base < total; base += BATCH * 128) {
+    uint4 a[BATCH], b[BATCH];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const double x1l = bf16_lo(aw[e]), x1h = bf16_hi(aw[e]);
-      const double x2l = bf16_lo(bw[e]), x2h = bf16_hi(bw[e]);
-      const double cl = cs[2 * e], sl = sn[2 * e], ch = cs[2 * e + 1], sh = sn[2 * e + 1];
-      const unsigned short r1l = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1l, cl), __dmul_rn(x2l, sl)));
-      const unsigned short r1h = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1h, ch), __dmul_rn(x2h, sh)));
-      const unsigned short r2l = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2l, cl), __dmul_rn(x1l, sl)));
-      const unsigned short r2h = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2h, ch), __dmul_rn(x1h, sh)));
-      y1[e] = (uint32_t)r1l | ((uint32_t)r1h << 16);
-      y2[e] = (uint32_t)r2l | ((uint32_t)r2h << 16);
+    for (int j = 0; j < BATCH; ++j) {
+      const int gi = base + j * 128;
+      if (gi >= total) break;
+      const int h = gi / GROUPS;
+      const __nv_bfloat16* src = h < Hq ? q + ((int64_t)t * Hq + h) * D
+                                        : k_in(k, t, Hkv, h - Hq, D);
+      a[j] = *reinterpret_cast<const uint4*>(src + i0);
+      b[j] = *reinterpret_cast<const uint4*>(src + HALF + i0);
     }
-    __nv_bfloat16* dst;
-    if (is_q) {
-      dst = q_rot + ((int64_t)t * Hq + h) * D;
-    } else {
-      if (!blk_ok) continue;
-      dst = cache.base + cache_offset(cache, blk, 0, h - Hq, slot);
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) {
+      const int gi = base + j * 128;
+      if (gi >= total) break;
+      const int h = gi / GROUPS;
+      const uint32_t aw[4] = {a[j].x, a[j].y, a[j].z, a[j].w};
+      const uint32_t bw[4] = {b[j].x, b[j].y, b[j].z, b[j].w};
+      uint32_t y1[4], y2[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const double x1l = bf16_lo(aw[e]), x1h = bf16_hi(aw[e]);
+        const double x2l = bf16_lo(bw[e]), x2h = bf16_hi(bw[e]);
+        const double cl = cs[2 * e], sl = sn[2 * e], ch = cs[2 * e + 1], sh = sn[2 * e + 1];
+        const unsigned short r1l = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1l, cl), __dmul_rn(x2l, sl)));
+        const unsigned short r1h = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1h, ch), __dmul_rn(x2h, sh)));
+        const unsigned short r2l = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2l, cl), __dmul_rn(x1l, sl)));
+        const unsigned short r2h = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2h, ch), __dmul_rn(x1h, sh)));
+        y1[e] = (uint32_t)r1l | ((uint32_t)r1h << 16);
+        y2[e] = (uint32_t)r2l | ((uint32_t)r2h << 16);
+      }
+      __nv_bfloat16* dst;
+      if (h < Hq) {
+        dst = q_rot + ((int64_t)t * Hq + h) * D;
+      } else {
+        if (!blk_ok) continue;
+        dst = cache.base + cache_offset(cache, blk, 0, h - Hq, slot);
+      }
+      *reinterpret_cast<uint4*>(dst + i0) = make_uint4(y1[0], y1[1], y1[2], y1[3]);
+      *reinterpret_cast<uint4*>(dst + HALF + i0) = make_uint4(y2[0], y2[1], y2[2], y2[3]);
     }
-    *reinterpret_cast<uint4*>(dst + i0) = make_uint4(y1[0], y1[1], y1[2], y1[3]);
-    *reinterpret_cast<uint4*>(dst + HALF + i0) = make_uint4(y2[0], y2[1], y2[2], y2[3]);
   }
   if (!blk_ok) return;
   constexpr int VCH = D / 8;
-  for (int ci = threadIdx.x; ci < Hkv * VCH; ci += blockDim.x) {
-    const int h = ci / VCH;
-    const int c8 = (ci - h * VCH) * 8;
-    const uint4 x = *reinterpret_cast<const uint4*>(v + ((int64_t)t * Hkv + h) * D + c8);
-    *reinterpret_cast<uint4*>(cache.base + cache_offset(cache, blk, 1, h, slot) + c8) = x;
+  const int nv = Hkv * VCH;
+  for (int base = threadIdx.x; base < nv; base += BATCH * 128) {
+    uint4 x[BATCH];
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) {
+      const int ci = base + j * 128;
+      if (ci >= nv) break;
+      const int h = ci / VCH;
+      x[j] = *reinterpret_cast<const uint4*>(v + ((int64_t)t * Hkv + h) * D + (ci - h * VCH) * 8);
+    }
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) {
+      const int ci = base + j * 128;
+      if (ci >= nv) break;
+      const int h = ci / VCH;
+      *reinterpret_cast<uint4*>(cache.base + cache_offset(cache, blk, 1, h, slot) + (ci - h * VCH) * 8) = x[j];
+    }
   }
 }
 

@@ -54,6 +54,7 @@ def lib() -> ctypes.CDLL:
         "fg_device_status": [V, V],
         "fg_attention_plan_info": [V, _c_int32_p],
         "fg_ragged_batch_set_timing": [V, I32],
+        "fg_ragged_batch_set_overlap": [V, I32],
         "fg_attention_kernel_ms": [V, _c_float_p],
         "fg_rotary_table": [D, I32, I32, I32, _c_float_p, _c_float_p],
     }
@@ -202,6 +203,9 @@ class RaggedBatch:
         keys = ("general_units", "decode_units", "tensor_units", "combine_groups", "partial_rows",
                 "launches")
         return dict(zip(keys, list(a)[:6]))
+
+    def set_overlap(self, enable: bool = True):
+        _check(lib().fg_ragged_batch_set_overlap(self._h, 1 if enable else 0), "fg_ragged_batch_set_overlap")
 
     def set_timing(self, enable: bool = True):
         _check(lib().fg_ragged_batch_set_timing(self._h, 1 if enable else 0), "fg_ragged_batch_set_timing")
