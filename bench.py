@@ -273,14 +273,23 @@ def run_fg(args, w, rank, ws, local_rank):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
 
+    host_parts = {"put": 0.0, "append": 0.0, "attention": 0.0}
+
     def step(ev):
         ev[0].record(stream)
+        t0 = time.perf_counter()
         batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, stream)
+        t1 = time.perf_counter()
         fg.rotary_kv_append(cache, batch, q, k, v, q_rot, w.n_q_heads, w.rope_theta, stream)
+        t2 = time.perf_counter()
         ev[1].record(stream)
         fg.ragged_attention(cache, batch, q_rot, out, w.n_q_heads, w.softmax_scale,
                             w.sliding_window, stream)
+        t3 = time.perf_counter()
         ev[2].record(stream)
+        host_parts["put"] += t1 - t0
+        host_parts["append"] += t2 - t1
+        host_parts["attention"] += t3 - t2
 
     def flush_l2():
         with torch.cuda.stream(stream):
@@ -297,6 +306,9 @@ def run_fg(args, w, rank, ws, local_rank):
     barrier()
     torch.cuda.synchronize()
     host_s = 0.0
+    for k_ in host_parts:
+        host_parts[k_] = 0.0
+    batch.host_profile_us(reset=True)
     with ClockSampler(local_rank) as clocks:
         for i in range(args.steps):
             t0 = time.perf_counter()
@@ -305,6 +317,7 @@ def run_fg(args, w, rank, ws, local_rank):
             flush_l2()
         torch.cuda.synchronize()
     barrier()
+    lib_host = {k_: v_ / args.steps for k_, v_ in batch.host_profile_us(reset=True).items()}
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
     put_append_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / len(evs)
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
@@ -383,6 +396,8 @@ def run_fg(args, w, rank, ws, local_rank):
                  "attention_call_ms": attn_ms_mean,
                  "put_append_ms": put_append_ms,
                  "host_enqueue_ms_per_step": 1000 * host_s / args.steps,
+                 "host_ms_per_call": {k_: 1000 * v_ / args.steps for k_, v_ in host_parts.items()},
+                 "library_host_us_per_step": lib_host,
                  "attention_call_GBps": work["attn_bytes"] / (attn_ms_mean / 1000) / 1e9,
                  "tc_TFLOPs": work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12 if kernel_ms["tc"] else None,
                  "step_roofline_ms": 1000 * max((work["attn_bytes"] + work["append_bytes"]) / (hbm * 1e9),

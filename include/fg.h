@@ -208,6 +208,14 @@ fg_status fg_attention_plan_info(const fg_ragged_batch* batch, int32_t info[8]);
 fg_status fg_ragged_batch_set_timing(fg_ragged_batch* batch, int32_t enable);
 fg_status fg_attention_kernel_ms(fg_ragged_batch* batch, float ms[4]);
 
+/* Host time spent inside this batch's calls, in microseconds, accumulated
+ * since the last reset: out[0] fg_ragged_batch_put in total, out[1] its
+ * validation, out[2] its wait for a free staging buffer, out[3]
+ * fg_ragged_attention in total, out[4] work planning, out[5] the wait for a
+ * free plan staging buffer, out[6] tensor-map encoding, out[7] kernel
+ * launches. reset != 0 zeroes the counters after reading them. */
+fg_status fg_host_profile_us(fg_ragged_batch* batch, double out[8], int32_t reset);
+
 /* Scheduling of one attention call that has both one-token decode units and
  * prompt-chunk query tiles. enable == 0 (default): the two kernels run one
  * after the other on the caller's stream, each with the whole GPU (two CTAs

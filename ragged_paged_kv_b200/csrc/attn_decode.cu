@@ -290,6 +290,11 @@ cudaError_t launch_decode_d(const CacheView& cache, const BatchView& batch, cons
     cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
+    // the largest shared-memory carveout, so CTAs of different kernels can
+    // share an SM
+    e = cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     configured = true;
   }
   attn_decode_kernel<D><<<n_items, C::kThreads, C::kSmem, stream>>>(cache, batch, items, q_rot, out,

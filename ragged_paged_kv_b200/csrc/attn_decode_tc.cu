@@ -50,8 +50,8 @@ struct DtcCfg {
   static constexpr int kOffBar = kOffRed + 2 * 4 * N * 4;
   // q_full, q_empty, slot_full[NSLOT], slot_empty[NSLOT], s_full[2], s_free[2],
   // p_full[2], pv_done[2], o_free, red_bar
-  static constexpr int kNumBars = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 1 + 1;
-  static constexpr int kSmem = kOffBar + kNumBars * 8 + 16;
+  static constexpr int kNumBars = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 1 + 1 + 2 * UnitQueue::kDepth;
+  static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + UnitQueue::kDepth * 4;
   static constexpr int kThreads = 192;
   static constexpr uint32_t kTmemCols = 64;
   static constexpr uint32_t kColS = 0;   // S^T buffers at columns 0 and 16
@@ -69,6 +69,7 @@ struct DtcArgs {
   int g;
   float scale_log2;
   int n_items;
+  int* counter;  // next-unit counter, zero at launch
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -131,7 +132,10 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
   uint64_t* pv_done = p_full + 2;
   uint64_t* o_free = pv_done + 2;
   uint64_t* red_bar = o_free + 1;  // rendezvous of the four softmax warps
+  uint64_t* uq_full = red_bar + 1;
+  uint64_t* uq_empty = uq_full + UnitQueue::kDepth;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  const UnitQueue uq{reinterpret_cast<int32_t*>(tmem_slot + 4), uq_full, uq_empty, 5};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = a.g;
@@ -152,6 +156,7 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
     }
     ptx::mbar_init(o_free, 4);
     ptx::mbar_init(red_bar, 4);
+    uq.init();
     ptx::fence_mbar_init();
   }
   if (warp == 5) {
@@ -171,7 +176,13 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
       const int BR = B < 64 ? B : 64;
       const int Hkv = a.cache.n_kv_heads;
       int gt = 0, un = 0;
-      for (int u = blockIdx.x; u < a.n_items && ok; u += gridDim.x, ++un) {
+      for (;; ++un) {
+        int u = -1;
+        if (!uq.push_next(un, a.counter, a.n_items, kWaitLimit, &u)) {
+          atomicOr(err, kErrTimeout);
+          ok = false;
+        }
+        if (u < 0 || !ok) break;
         const WorkItem it = a.items[u];
         const int s = it.seq, h = it.kv_head;
         const int row = a.batch.cu_q[s] + it.tok_begin;
@@ -240,7 +251,13 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
         ptx::mma_commit(&pv_done[pb]);
         ptx::mma_commit(&slot_empty[slot]);
       };
-      for (int u = blockIdx.x; u < a.n_items && ok; u += gridDim.x, ++un) {
+      for (;; ++un) {
+        int u = -1;
+        if (!uq.pop(un, false, kWaitLimit, &u)) {
+          atomicOr(err, kErrTimeout);
+          ok = false;
+        }
+        if (u < 0 || !ok) break;
         const WorkItem it = a.items[u];
         const int k00 = it.key_begin - (it.key_begin & 63);
         const int n_st = (it.key_end - k00 + C::BK - 1) / C::BK;
@@ -279,7 +296,13 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
       return wait_or_flag(red_bar, (red_phase++) & 1, err, ok);
     };
     int gt = 0, un = 0;
-    for (int u = blockIdx.x; u < a.n_items && ok; u += gridDim.x, ++un) {
+    for (;; ++un) {
+      int u = -1;
+      if (!uq.pop(un, true, kWaitLimit, &u)) {
+        if (lane == 0) atomicOr(err, kErrTimeout);
+        ok = false;
+      }
+      if (u < 0 || !ok) break;
       const WorkItem it = a.items[u];
       const int s = it.seq;
       const int ctx = a.batch.ctx[s];
@@ -432,16 +455,22 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
 cudaError_t launch_attention_decode_tc(const void* tm_q1, const void* tm_kv, const CacheView& cache,
                                        const BatchView& batch, const WorkItem* items, int n_items,
                                        __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
-                                       int g, float scale_log2, int grid, cudaStream_t stream) {
+                                       int g, float scale_log2, int grid, int* counter,
+                                       cudaStream_t stream) {
   if (n_items == 0) return cudaSuccess;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          DtcCfg::kSmem);
     if (e != cudaSuccess) return e;
+    // the largest shared-memory carveout, so CTAs of different kernels can
+    // share an SM
+    e = cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     configured = true;
   }
-  DtcArgs args{cache, batch, items, out, part_o, part_ml, n_q_heads, g, scale_log2, n_items};
+  DtcArgs args{cache, batch, items, out, part_o, part_ml, n_q_heads, g, scale_log2, n_items, counter};
   grid = grid < 1 ? 1 : (grid > n_items ? n_items : grid);
   attn_decode_tc_kernel<<<grid, DtcCfg::kThreads, DtcCfg::kSmem, stream>>>(
       *static_cast<const CUtensorMap*>(tm_q1), *static_cast<const CUtensorMap*>(tm_kv), args);

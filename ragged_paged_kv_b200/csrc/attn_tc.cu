@@ -53,8 +53,8 @@ struct TcCfg {
   static constexpr int kOffBar = kOffP + kPBytes;
   // q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST],
   // s_full[2], s_free[2], p_full, pv_done, o_free
-  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + 2 + 2 + 3;
-  static constexpr int kSmem = kOffBar + kNumBars * 8 + 16;
+  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + 2 + 2 + 3 + 2 * UnitQueue::kDepth;
+  static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + UnitQueue::kDepth * 4;
   static constexpr int kThreads = 192;
   static constexpr uint32_t kTmemCols = 256;
   static constexpr uint32_t kColS = 0;     // S buffers at columns 0 and BN
@@ -74,6 +74,7 @@ struct TcArgs {
   float scale_log2;
   int window;
   int n_items;
+  int* counter;  // next-unit counter, zero at launch
 };
 
 // What every role needs to know about one unit.
@@ -144,7 +145,12 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
   uint64_t* p_full = s_free + 2;
   uint64_t* pv_done = p_full + 1;
   uint64_t* o_free = pv_done + 1;
+  uint64_t* uq_full = o_free + 1;
+  uint64_t* uq_empty = uq_full + UnitQueue::kDepth;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  // units come from a global counter through this queue (MMA thread and the
+  // four softmax warps consume)
+  const UnitQueue uq{reinterpret_cast<int32_t*>(tmem_slot + 4), uq_full, uq_empty, 5};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = a.g;
@@ -168,6 +174,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
     ptx::mbar_init(p_full, 4);
     ptx::mbar_init(pv_done, 1);
     ptx::mbar_init(o_free, 4);
+    uq.init();
     ptx::fence_mbar_init();
   }
   if (warp == 5) {
@@ -187,7 +194,13 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
       const int BR = B < 64 ? B : 64;
       const int Hkv = a.cache.n_kv_heads;
       int gt = 0, un = 0;
-      for (int u = blockIdx.x; u < a.n_items && ok; u += gridDim.x, ++un) {
+      for (;; ++un) {
+        int u = -1;
+        if (!uq.push_next(un, a.counter, a.n_items, kWaitLimit, &u)) {
+          atomicOr(err, kErrTimeout);
+          ok = false;
+        }
+        if (u < 0 || !ok) break;
         const Unit x = load_unit(a, u, C::BN);
         if (un >= 1 && !wait_or_flag(q_empty, (un - 1) & 1, err, ok)) break;
         ptx::mbar_arrive_expect_tx(q_full, C::kQBytes);
@@ -267,7 +280,13 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
         ptx::mma_commit(pv_done);
         ptx::mma_commit(&v_empty[vs]);
       };
-      for (int u = blockIdx.x; u < a.n_items && ok; u += gridDim.x, ++un) {
+      for (;; ++un) {
+        int u = -1;
+        if (!uq.pop(un, false, kWaitLimit, &u)) {
+          atomicOr(err, kErrTimeout);
+          ok = false;
+        }
+        if (u < 0 || !ok) break;
         const Unit x = load_unit(a, u, C::BN);
         if (!wait_or_flag(q_full, un & 1, err, ok)) break;
         const int gt0 = gt;
@@ -297,7 +316,13 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
     const int r = threadIdx.x;  // query row == TMEM lane
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     int gt = 0, un = 0;
-    for (int u = blockIdx.x; u < a.n_items && ok; u += gridDim.x, ++un) {
+    for (;; ++un) {
+      int u = -1;
+      if (!uq.pop(un, true, kWaitLimit, &u)) {
+        if (lane == 0) atomicOr(err, kErrTimeout);
+        ok = false;
+      }
+      if (u < 0 || !ok) break;
       const Unit x = load_unit(a, u, C::BN);
       const bool row_ok = r < x.R;
       const int p_r = x.ctx + x.tok_begin + r / g;
@@ -468,18 +493,31 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
   }
 }
 
+// Dynamic shared memory requested when the kernel must leave each SM to one
+// CTA of its own beside one decode CTA: two CTAs of this size (plus the 1 KB
+// each CTA reserves) exceed an SM's 228 KB, one of them plus a decode CTA
+// does not.
+constexpr int kTcSmemExclusive = 117760;
+
 template <int D>
 cudaError_t launch_tc_d(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const TcArgs& args,
-                        int grid, cudaStream_t stream) {
+                        int grid, bool exclusive, cudaStream_t stream) {
   using C = TcCfg<D>;
+  static_assert(C::kSmem <= kTcSmemExclusive, "padding below the kernel's own need");
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmem);
+                                         kTcSmemExclusive);
+    if (e != cudaSuccess) return e;
+    // the largest shared-memory carveout, so CTAs of different kernels can
+    // share an SM
+    e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  attn_tc_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tm_q, tm_kv, args);
+  attn_tc_kernel<D><<<grid, C::kThreads, exclusive ? kTcSmemExclusive : C::kSmem, stream>>>(tm_q, tm_kv,
+                                                                                          args);
   return cudaGetLastError();
 }
 
@@ -488,15 +526,16 @@ cudaError_t launch_tc_d(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const
 cudaError_t launch_attention_tc(const void* tm_q, const void* tm_kv, const CacheView& cache,
                                 const BatchView& batch, const WorkItem* items, int n_items,
                                 __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
-                                int g, float scale_log2, int window, int grid,
-                                cudaStream_t stream) {
+                                int g, float scale_log2, int window, int grid, bool exclusive,
+                                int* counter, cudaStream_t stream) {
   if (n_items == 0) return cudaSuccess;
-  TcArgs args{cache, batch, items, out, part_o, part_ml, n_q_heads, g, scale_log2, window, n_items};
+  TcArgs args{cache, batch, items, out, part_o, part_ml, n_q_heads, g, scale_log2, window, n_items,
+              counter};
   grid = grid < 1 ? 1 : (grid > n_items ? n_items : grid);
   const CUtensorMap& q = *static_cast<const CUtensorMap*>(tm_q);
   const CUtensorMap& kv = *static_cast<const CUtensorMap*>(tm_kv);
-  if (cache.head_dim == 128) return launch_tc_d<128>(q, kv, args, grid, stream);
-  return launch_tc_d<64>(q, kv, args, grid, stream);
+  if (cache.head_dim == 128) return launch_tc_d<128>(q, kv, args, grid, exclusive, stream);
+  return launch_tc_d<64>(q, kv, args, grid, exclusive, stream);
 }
 
 }  // namespace fg

@@ -6,6 +6,7 @@
 // asynchronous host-to-device copy; fg_ragged_attention plans its work units
 // on the host (integer work only) and sends them the same way.
 #include <algorithm>
+#include <chrono>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -50,6 +51,11 @@ fg_status cuda_fail(cudaError_t e, const char* what) {
   } while (0)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+double now_us() {
+  return std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now().time_since_epoch())
+      .count();
+}
 
 // A pinned host staging area with two halves used in turn; before a half is
 // rewritten the host waits for the copy that last read it.
@@ -127,6 +133,7 @@ struct fg_ragged_batch {
   int32_t* dmeta = nullptr;
   size_t dmeta_words = 0;
   int32_t* derr = nullptr;
+  int32_t* dctr = nullptr;  // next-unit counters of the persistent kernels
   Staging meta_stage;
   // last put
   const fg_kv_cache* cache = nullptr;
@@ -152,6 +159,9 @@ struct fg_ragged_batch {
   bool timing = false;
   cudaEvent_t tev[8] = {};
   bool tran[4] = {};
+  // host-time profile (microseconds, accumulated): put, validation, put
+  // staging wait, attention, planning, plan staging wait, tensor maps, calls
+  double hprof[8] = {};
   // split-KV partials
   float* ws = nullptr;
   size_t ws_bytes = 0;
@@ -320,6 +330,7 @@ extern "C" fg_status fg_ragged_batch_destroy(fg_ragged_batch* b) {
   b->plan_stage.release();
   if (b->dmeta) cudaFree(b->dmeta);
   if (b->derr) cudaFree(b->derr);
+  if (b->dctr) cudaFree(b->dctr);
   if (b->dplan) cudaFree(b->dplan);
   if (b->ws) cudaFree(b->ws);
   for (cudaEvent_t e : b->tev)
@@ -430,9 +441,11 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
                                          const int32_t* ids, const int32_t* ql, const int32_t* cl,
                                          const int32_t* bt, int32_t stride, void* stream) {
   if (!b || !c) return fail(FG_ERR_INVALID_ARG, "NULL handle");
+  const double t_in = now_us();
   int64_t T = 0, nblk = 0;
   int32_t maxpos = -1;
   fg_status st = validate_batch(b, c, S, ids, ql, cl, bt, stride, &T, &nblk, &maxpos);
+  b->hprof[1] += now_us() - t_in;
   if (st) {
     b->cache = nullptr;  // the previous batch is no longer valid either
     return st;
@@ -444,6 +457,7 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
     FG_CUDA(cudaGetDevice(&b->device));
     FG_CUDA(cudaMalloc(&b->dmeta, b->dmeta_words * 4));
     FG_CUDA(cudaMalloc(&b->derr, 4));
+    FG_CUDA(cudaMalloc(&b->dctr, 64));
     FG_CUDA(cudaMemset(b->derr, 0, 4));
     st = b->meta_stage.reserve(b->dmeta_words * 4);
     if (st) return st;
@@ -452,7 +466,9 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
   const size_t words = 3 * (size_t)S + 2 + (size_t)T + (size_t)nblk;
   void* hp = nullptr;
   int slot = 0;
+  const double t_w = now_us();
   st = b->meta_stage.acquire(&hp, &slot);
+  b->hprof[2] += now_us() - t_w;
   if (st) return st;
   int32_t* h = static_cast<int32_t*>(hp);
   int32_t* cu = h;
@@ -473,6 +489,7 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
   }
   st = b->meta_stage.copy(slot, b->dmeta, words * 4, strm);
   if (st) return st;
+  b->hprof[0] += now_us() - t_in;
   int32_t* d = b->dmeta;
   b->view.cu_q = d;
   b->view.ctx = d + S + 1;
@@ -632,7 +649,10 @@ fg_status prepare_plan(fg_ragged_batch* b, const fg_kv_cache* c, int32_t g, int3
   const uint64_t key[4] = {b->put_gen, (uint64_t)g, (uint64_t)(uint32_t)window,
                            (uint64_t)c->head_dim | ((uint64_t)use_tc << 32)};
   if (std::equal(key, key + 4, b->plan_key) && b->dplan) return FG_OK;
-  fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc, &b->plan);
+  const double t_p = now_us();
+  fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc,
+                 2 * sm_count(), &b->plan);
+  b->hprof[4] += now_us() - t_p;
   const size_t bytes = b->plan.bytes();
   if (bytes > b->dplan_bytes) {
     if (b->dplan) FG_CUDA(cudaFreeAsync(b->dplan, strm));
@@ -645,7 +665,9 @@ fg_status prepare_plan(fg_ragged_batch* b, const fg_kv_cache* c, int32_t g, int3
   if (st) return st;
   void* hp = nullptr;
   int slot = 0;
+  const double t_w = now_us();
   st = b->plan_stage.acquire(&hp, &slot);
+  b->hprof[5] += now_us() - t_w;
   if (st) return st;
   b->plan.pack(hp);
   st = b->plan_stage.copy(slot, b->dplan, bytes, strm);
@@ -699,11 +721,14 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   const bool use_tc = tc_eligible(const_cast<fg_kv_cache*>(c), g);
   if (!use_tc && g > fg::kMaxGroup)
     return fail(FG_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads = %d > %d", g, fg::kMaxGroup);
+  const double t_a = now_us();
   CUtensorMap tm_q, tm_q1;
   if (use_tc && (!make_q_map(&tm_q, q_rot, b->n_tokens, n_q_heads, c->head_dim, g) ||
                  !make_q_map(&tm_q1, q_rot, b->n_tokens, n_q_heads, c->head_dim, g, 1)))
     return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q_rot");
+  b->hprof[6] += now_us() - t_a;
   st = prepare_plan(b, c, g, window, use_tc, strm);
+  const double t_l = now_us();
   if (st) return st;
   const fg::Plan& P = b->plan;
   const size_t need = (size_t)P.part_rows * (c->head_dim + 2);
@@ -746,16 +771,20 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   if (both) {
     st = ensure_aux_stream(b);
     if (st) return st;
+    tc_stream = b->aux;
+  }
+  // the persistent kernels' unit counters start at zero
+  if (P.n_tc || P.n_dtc) FG_CUDA(cudaMemsetAsync(b->dctr, 0, 8, strm));
+  if (both) {
     FG_CUDA(cudaEventRecord(b->fork, strm));
     FG_CUDA(cudaStreamWaitEvent(b->aux, b->fork, 0));
-    tc_stream = b->aux;
   }
   if (P.n_tc) {
     if ((st = mark(1, 0, tc_stream))) return st;
     e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
                                 part_ml, n_q_heads, g, scale_log2, window, tc_grid(P, b->overlap),
-                                tc_stream);
+                                both, b->dctr, tc_stream);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
     if ((st = mark(1, 1, tc_stream))) return st;
   }
@@ -770,7 +799,7 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
     e = fg::launch_attention_decode_tc(&tm_q1, &c->tm_kv, cv, b->view,
                                        reinterpret_cast<const WorkItem*>(base + P.off_dtc), P.n_dtc, o,
                                        part_o, part_ml, n_q_heads, g, scale_log2,
-                                       sm_count() * (both ? 1 : 2), strm);
+                                       sm_count() * (both ? 1 : 2), b->dctr + 1, strm);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core decode launch");
     if ((st = mark(0, 1, strm))) return st;
   }
@@ -784,6 +813,18 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
                          c->head_dim, strm);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   if (P.n_combine && (st = mark(3, 1, strm))) return st;
+  const double t_end = now_us();
+  b->hprof[7] += t_end - t_l;
+  b->hprof[3] += t_end - t_a;
+  return FG_OK;
+}
+
+extern "C" fg_status fg_host_profile_us(fg_ragged_batch* b, double out[8], int32_t reset) {
+  if (!b || !out) return fail(FG_ERR_INVALID_ARG, "NULL argument");
+  for (int i = 0; i < 8; ++i) {
+    out[i] = b->hprof[i];
+    if (reset) b->hprof[i] = 0.0;
+  }
   return FG_OK;
 }
 
@@ -885,10 +926,13 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
     return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q_rot");
   thread_local fg::Plan P;
   thread_local std::vector<unsigned char> packed;
-  fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc, &P);
-  if (P.bytes() > plan_bytes)
+  fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc,
+                 2 * sm_count(), &P);
+  // the last 256 bytes of the plan area hold the persistent kernels' counters
+  if (P.bytes() + 256 > plan_bytes)
     return fail(FG_ERR_CAPACITY, "pass needs a %zu-byte work plan, the fixed area holds %zu",
-                P.bytes(), plan_bytes);
+                P.bytes(), plan_bytes - 256);
+  int* ctr = reinterpret_cast<int*>(static_cast<char*>(plan_dev) + plan_bytes - 256);
   const size_t need = (size_t)P.part_rows * (c->head_dim + 2);
   if (need > ws_floats)
     return fail(FG_ERR_CAPACITY, "pass needs %zu split-workspace floats, the fixed area holds %zu",
@@ -897,6 +941,7 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
   P.pack(packed.data());
   if (!packed.empty())
     FG_CUDA(cudaMemcpyAsync(plan_dev, packed.data(), packed.size(), cudaMemcpyHostToDevice, strm));
+  if (P.n_tc || P.n_dtc) FG_CUDA(cudaMemsetAsync(ctr, 0, 8, strm));
   float* part_o = ws;
   float* part_ml = ws + (size_t)P.part_rows * c->head_dim;
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
@@ -914,13 +959,15 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
   if (P.n_tc) {
     e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
-                                part_ml, n_q_heads, g, scale_log2, window, 2 * sm_count(), strm);
+                                part_ml, n_q_heads, g, scale_log2, window, 2 * sm_count(), false,
+                                ctr, strm);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
   }
   if (P.n_dtc) {
     e = fg::launch_attention_decode_tc(&tm_q1, &c->tm_kv, cv, b->view,
                                        reinterpret_cast<const WorkItem*>(base + P.off_dtc), P.n_dtc, o,
-                                       part_o, part_ml, n_q_heads, g, scale_log2, 2 * sm_count(), strm);
+                                       part_o, part_ml, n_q_heads, g, scale_log2, 2 * sm_count(), ctr + 1,
+                                       strm);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core decode launch");
   }
   e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),

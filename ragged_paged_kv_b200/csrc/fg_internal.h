@@ -83,17 +83,21 @@ cudaError_t launch_attention_decode(const CacheView& cache, const BatchView& bat
                                     cudaStream_t stream);
 
 // tm_q / tm_kv point to CUtensorMap objects (host memory, passed by value).
+// The persistent tensor-core kernels take their units from *counter, which
+// must be zero when the kernel starts.
 cudaError_t launch_attention_tc(const void* tm_q, const void* tm_kv, const CacheView& cache,
                                 const BatchView& batch, const WorkItem* items, int n_items,
                                 __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
-                                int g, float scale_log2, int window, int grid, cudaStream_t stream);
+                                int g, float scale_log2, int window, int grid, bool exclusive,
+                                int* counter, cudaStream_t stream);
 
 // Grouped (or MHA) one-token decode on tensor cores, keys as MMA rows;
 // tm_q1 views q_rot with boxes of 64 dims x g heads x 1 token. d = 128.
 cudaError_t launch_attention_decode_tc(const void* tm_q1, const void* tm_kv, const CacheView& cache,
                                        const BatchView& batch, const WorkItem* items, int n_items,
                                        __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
-                                       int g, float scale_log2, int grid, cudaStream_t stream);
+                                       int g, float scale_log2, int grid, int* counter,
+                                       cudaStream_t stream);
 
 cudaError_t launch_combine(const BatchView& batch, const CombineItem* items, int n_items,
                            int max_rows, const float* part_o, const float* part_ml,

@@ -17,8 +17,7 @@ void Plan::pack(void* dst) const {
 }
 
 void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& ctx_lens,
-                int n_kv_heads, int g, int head_dim, int window, bool use_tc, Plan* out) {
-  (void)head_dim;
+                int n_kv_heads, int g, int head_dim, int window, bool use_tc, int slots, Plan* out) {
   Plan& P = *out;
   P.general.clear();
   P.decode.clear();
@@ -29,47 +28,71 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
   P.max_combine_rows = 0;
   const int tok_per_tile = std::max(1, kGeneralRows / g);
   const int S = (int)q_lens.size();
-  // Append units for one (seq, kv head, token tile) over keys [kb, ke) to
-  // `list`, split on `split`-key boundaries of absolute position.
-  auto emit = [&](std::vector<WorkItem>& list, int s, int h, int t0, int nt, int kb, int ke,
-                  int split) {
+  int dense_split = 0;  // pieces per long query tile, decided on first use
+  // Append the units of one (seq, token tile) over keys [kb, ke) for every kv
+  // head to `list`, split on `split`-key boundaries of absolute position.
+  // The split ranges are computed once and repeated per head.
+  int32_t rng[2 * 64];
+  auto emit = [&](std::vector<WorkItem>& list, int s, int t0, int nt, int kb, int ke, int split) {
     const int R = nt * g;
     const int kb_al = kb - (kb % 64);
-    const int n = (ke - kb_al + split - 1) / split;
+    const int n = std::min(64, (ke - kb_al + split - 1) / split);
     if (n <= 1) {
-      list.push_back(WorkItem{s, h, t0, nt, kb, ke, -1, R});
+      for (int h = 0; h < n_kv_heads; ++h) list.push_back(WorkItem{s, h, t0, nt, kb, ke, -1, R});
       return;
     }
-    const int base = P.part_rows;
-    for (int i = 0; i < n; ++i) {
-      const int lo = i == 0 ? kb : kb_al + i * split;
-      const int hi = std::min(ke, kb_al + (i + 1) * split);
-      list.push_back(WorkItem{s, h, t0, nt, lo, hi, base + i * R, R});
+    const int sp = (ke - kb_al + n - 1) / n;  // never more than 64 pieces
+    const int step = std::max(split, (sp + 63) & ~63);
+    int m = 0;
+    for (int lo = kb; lo < ke; ++m) {
+      const int hi = std::min(ke, kb_al + (m + 1) * step);
+      rng[2 * m] = lo;
+      rng[2 * m + 1] = hi;
+      lo = hi;
     }
-    P.part_rows += n * R;
-    P.combine.push_back(CombineItem{s, h, t0, nt, base, n, R, 0});
+    for (int h = 0; h < n_kv_heads; ++h) {
+      const int base = P.part_rows;
+      for (int i = 0; i < m; ++i) list.push_back(WorkItem{s, h, t0, nt, rng[2 * i], rng[2 * i + 1], base + i * R, R});
+      P.part_rows += m * R;
+      P.combine.push_back(CombineItem{s, h, t0, nt, base, m, R, 0});
+    }
     P.max_combine_rows = std::max(P.max_combine_rows, R);
   };
   for (int s = 0; s < S; ++s) {
     const int q = q_lens[s], c = ctx_lens[s];
     if (use_tc && q == 1 && head_dim == 128 && g <= kDtcMaxGroup) {
       const int kb = window > 0 ? std::max(0, c - window + 1) : 0;
-      for (int h = 0; h < n_kv_heads; ++h) emit(P.dtc, s, h, 0, 1, kb, c + 1, kTcDecodeSplitKeys);
+      emit(P.dtc, s, 0, 1, kb, c + 1, kTcDecodeSplitKeys);
       continue;
     }
     if (q == 1 && g == 1) {
       const int kb = window > 0 ? std::max(0, c - window + 1) : 0;
-      for (int h = 0; h < n_kv_heads; ++h) emit(P.decode, s, h, 0, 1, kb, c + 1, kDecodeSplitKeys);
+      emit(P.decode, s, 0, 1, kb, c + 1, kDecodeSplitKeys);
       continue;
     }
     if (use_tc) {
       const int tpt = kTcRows / g;
+      // Few long query tiles leave persistent CTAs idle at the end: then
+      // tiles of >= 2 * kTcMinSplitKeys keys are cut into pieces of at least
+      // kTcMinSplitKeys keys so that there are about 4 units per CTA slot.
+      if (dense_split == 0) {
+        long long n_dense = 0;
+        for (int s2 = 0; s2 < S; ++s2)
+          if (!(q_lens[s2] == 1 && head_dim == 128 && g <= kDtcMaxGroup))
+            n_dense += (q_lens[s2] + tpt - 1) / tpt;
+        n_dense *= n_kv_heads;
+        dense_split = n_dense > 0 && n_dense < 4LL * slots ? (int)((4LL * slots + n_dense - 1) / n_dense) : 1;
+        dense_split = std::min(dense_split, 8);
+      }
       for (int t0 = 0; t0 < q; t0 += tpt) {
         const int nt = std::min(tpt, q - t0);
         const int p0 = c + t0, p1 = c + t0 + nt - 1;
         const int kb = window > 0 ? std::max(0, p0 - window + 1) : 0;
-        const int split = nt * g <= 16 ? kTcDecodeSplitKeys : (1 << 30);
-        for (int h = 0; h < n_kv_heads; ++h) emit(P.tc, s, h, t0, nt, kb, p1 + 1, split);
+        int split = nt * g <= 16 ? kTcDecodeSplitKeys : (1 << 30);
+        const int nk = p1 + 1 - kb;
+        if (nt * g > 16 && dense_split > 1 && nk >= 2 * kTcMinSplitKeys)
+          split = std::max(kTcMinSplitKeys, ((nk + dense_split - 1) / dense_split + 63) & ~63);
+        emit(P.tc, s, t0, nt, kb, p1 + 1, split);
       }
       continue;
     }
@@ -77,18 +100,34 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
       const int nt = std::min(tok_per_tile, q - t0);
       const int p0 = c + t0, p1 = c + t0 + nt - 1;
       const int kb = window > 0 ? std::max(0, p0 - window + 1) : 0;
-      for (int h = 0; h < n_kv_heads; ++h) emit(P.general, s, h, t0, nt, kb, p1 + 1, kSplitKeys);
+      emit(P.general, s, t0, nt, kb, p1 + 1, kSplitKeys);
     }
   }
-  // longest units first, so the hardware block scheduler ends the grid evenly
-  std::stable_sort(P.decode.begin(), P.decode.end(), [](const WorkItem& a, const WorkItem& b) {
-    return a.key_end - a.key_begin > b.key_end - b.key_begin;
-  });
-  auto longest_first = [](const WorkItem& a, const WorkItem& b) {
-    return a.key_end - a.key_begin > b.key_end - b.key_begin;
+  // longest units first (by 64-key stages), stable: a counting sort, so
+  // planning stays linear in the number of units
+  auto by_length = [&P](std::vector<WorkItem>& v) {
+    if (v.size() < 2) return;
+    constexpr int kBuckets = 4096;
+    auto stages = [](const WorkItem& w) {
+      const int n = (w.key_end - (w.key_begin - (w.key_begin & 63)) + 63) >> 6;
+      return n < kBuckets - 1 ? n : kBuckets - 1;
+    };
+    std::vector<int32_t>& cnt = P.sort_count;
+    cnt.assign(kBuckets + 1, 0);
+    for (const WorkItem& w : v) ++cnt[kBuckets - 1 - stages(w)];
+    int32_t run = 0;
+    for (int b = 0; b <= kBuckets; ++b) {
+      const int32_t c = cnt[b];
+      cnt[b] = run;
+      run += c;
+    }
+    P.sort_tmp.resize(v.size());
+    for (const WorkItem& w : v) P.sort_tmp[cnt[kBuckets - 1 - stages(w)]++] = w;
+    v.swap(P.sort_tmp);
   };
-  std::stable_sort(P.tc.begin(), P.tc.end(), longest_first);
-  std::stable_sort(P.dtc.begin(), P.dtc.end(), longest_first);
+  by_length(P.decode);
+  by_length(P.tc);
+  by_length(P.dtc);
   P.n_general = (int32_t)P.general.size();
   P.n_decode = (int32_t)P.decode.size();
   P.n_tc = (int32_t)P.tc.size();

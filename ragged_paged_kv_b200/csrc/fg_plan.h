@@ -16,6 +16,7 @@ constexpr int kDecodeSplitKeys = 512;  // keys per unit of the MHA decode kernel
 constexpr int kTcRows = 128;           // query rows per tensor-core tile
 constexpr int kTcDecodeSplitKeys = 2048;  // keys per unit for small (decode) tc tiles
 constexpr int kDtcMaxGroup = 16;          // q heads per kv head the decode tc kernel serves
+constexpr int kTcMinSplitKeys = 4096;     // shortest piece when a long query tile is split
 
 struct Plan {
   std::vector<WorkItem> general;   // CUDA-core general path
@@ -23,6 +24,8 @@ struct Plan {
   std::vector<WorkItem> tc;        // tensor-core query tiles (prompt chunks)
   std::vector<WorkItem> dtc;       // one-token decodes on tensor cores (keys as MMA rows)
   std::vector<CombineItem> combine;
+  std::vector<WorkItem> sort_tmp;  // scratch of the longest-first sort
+  std::vector<int32_t> sort_count;
   int32_t part_rows = 0;         // partial rows the split units write
   int32_t max_combine_rows = 0;  // largest n_rows among combine items
   // packed device layout (bytes from the plan buffer's start)
@@ -44,7 +47,8 @@ struct Plan {
 // go to the keys-as-rows decode kernel (dtc), other tokens to 128-row query
 // tiles (tc); without it, MHA decodes go to the CUDA-core decode kernel and
 // the rest to the general path.
+// slots: CTAs the persistent kernels run with (for the long-tile split).
 void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& ctx_lens,
-                int n_kv_heads, int g, int head_dim, int window, bool use_tc, Plan* out);
+                int n_kv_heads, int g, int head_dim, int window, bool use_tc, int slots, Plan* out);
 
 }  // namespace fg

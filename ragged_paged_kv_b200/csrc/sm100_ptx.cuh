@@ -167,4 +167,49 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
 }
 
 }  // namespace ptx
+
+// Dynamic work distribution inside a persistent CTA: one scheduling thread
+// takes the next unit index from a global counter (longest units first, so
+// this is greedy longest-processing-time scheduling) and hands it to the
+// CTA's other roles through a small shared-memory queue guarded by
+// mbarriers. -1 means no work is left.
+struct UnitQueue {
+  static constexpr int kDepth = 4;
+  int32_t* idx;     // shared [kDepth]
+  uint64_t* full;   // shared [kDepth], one arrival (the scheduler)
+  uint64_t* empty;  // shared [kDepth], one arrival per consumer
+  int n_consumers;
+
+  __device__ void init() const {
+    for (int i = 0; i < kDepth; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], n_consumers);
+    }
+  }
+  // Scheduler side; returns false if a bounded wait gave up.
+  __device__ bool push_next(int un, int* counter, int n_units, long long limit, int* out) const {
+    const int slot = un % kDepth;
+    if (un >= kDepth && !ptx::mbar_wait_bounded(&empty[slot], ((un / kDepth) - 1) & 1, limit)) return false;
+    const int v = atomicAdd(counter, 1);
+    *out = v < n_units ? v : -1;
+    idx[slot] = *out;
+    ptx::mbar_arrive(&full[slot]);
+    return true;
+  }
+  // Consumer side. A whole warp calls it with warp_wide = true (its lane 0
+  // arrives once all lanes have read); a lone thread with warp_wide = false.
+  __device__ bool pop(int un, bool warp_wide, long long limit, int* out) const {
+    const int slot = un % kDepth;
+    if (!ptx::mbar_wait_bounded(&full[slot], (un / kDepth) & 1, limit)) return false;
+    *out = idx[slot];
+    if (warp_wide) {
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&empty[slot]);
+    } else {
+      ptx::mbar_arrive(&empty[slot]);
+    }
+    return true;
+  }
+};
+
 }  // namespace fg

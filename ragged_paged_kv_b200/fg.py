@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
         "fg_attention_plan_info": [V, _c_int32_p],
         "fg_ragged_batch_set_timing": [V, I32],
         "fg_ragged_batch_set_overlap": [V, I32],
+        "fg_host_profile_us": [V, ctypes.POINTER(ctypes.c_double), I32],
         "fg_attention_kernel_ms": [V, _c_float_p],
         "fg_rotary_table": [D, I32, I32, I32, _c_float_p, _c_float_p],
     }
@@ -203,6 +204,13 @@ class RaggedBatch:
         keys = ("general_units", "decode_units", "tensor_units", "combine_groups", "partial_rows",
                 "launches")
         return dict(zip(keys, list(a)[:6]))
+
+    def host_profile_us(self, reset: bool = False) -> dict:
+        a = (ctypes.c_double * 8)()
+        _check(lib().fg_host_profile_us(self._h, a, 1 if reset else 0), "fg_host_profile_us")
+        keys = ("put", "put_validate", "put_stage_wait", "attention", "plan", "plan_stage_wait",
+                "tensor_maps", "launches")
+        return dict(zip(keys, list(a)))
 
     def set_overlap(self, enable: bool = True):
         _check(lib().fg_ragged_batch_set_overlap(self._h, 1 if enable else 0), "fg_ragged_batch_set_overlap")

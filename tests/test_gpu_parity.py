@@ -243,3 +243,26 @@ def test_chunked_prefill_equals_one_shot_70b_shape():
                                             one.softmax_scale)[0]
     assert_close(bf16_to_f64(out1[tok]), ref[tok], "one-shot vs oracle")
     _free(c1, c2)
+
+
+def test_overlapped_schedule_gives_bit_identical_output():
+    """Running the query-tile kernel beside the decode kernel on a second
+    stream changes only which CTA takes which unit: same bits out."""
+    for w in (W.config2(), W.config5()):
+        outs = []
+        for overlap in (False, True):
+            cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+            fixtures.fill(cache.tensor)
+            fixtures.write_context(w, cache.tensor, keep=(), others="pool")
+            batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+            batch.set_overlap(overlap)
+            batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables)
+            q, k, v = fixtures.qkv_device(w)
+            q_rot, out = torch.empty_like(q), torch.empty_like(q)
+            fg.forward(cache, batch, q, k, v, q_rot, out, w.n_q_heads, w.rope_theta, w.softmax_scale,
+                       w.sliding_window)
+            torch.cuda.synchronize()
+            batch.device_status()
+            outs.append(to_bits(out))
+            _free(cache, batch)
+        assert np.array_equal(outs[0], outs[1]), w.name
