@@ -3,26 +3,29 @@
 // A work unit is one 128-row query tile of one sequence and kv head: the
 // rows are (token, q head of the group) pairs, 128/g consecutive new tokens
 // times the g q heads that share the kv head, so a grouped-query tile reuses
-// each K/V tile for all g heads. Prompt chunks give full tiles; a grouped
-// decode token gives a g-row tile. The kernel is persistent: CTA b takes
-// units b, b + grid, ... of a longest-first list, and every role counts
-// tiles globally, so the rings and barrier phases run on across units (the
-// next unit's K/V stream in while the last one's epilogue runs). A unit walks
-// its key range in 64-key tiles:
+// each K/V tile for all g heads. The kernel is persistent: the TMA warp takes
+// units one by one from a global counter over a longest-first list and hands
+// them to the other warps, and every role counts tiles globally, so the rings
+// and barrier phases run on across units (the next unit's K/V stream in while
+// the last one's epilogue runs). A unit walks its key range in 64-key tiles:
 //
 //   warp 4 (TMA)      Q once (3-D box: 64 dims x g heads x 128/g tokens), then
 //                     K and V tiles through the block table, one 2-D box per
 //                     (block part, 64 dims), into 2-stage K and V rings;
-//   warp 5 (MMA)      one thread issues S = Q K^T into a double-buffered TMEM
-//                     S tile, and O += P V into a TMEM O tile;
+//   warp 5 (MMA)      one thread issues S = Q K^T into one of two TMEM S
+//                     tiles, and O += P V into the TMEM O tile with P read
+//                     from tensor memory;
 //   warps 0-3         thread r owns query row r (TMEM lane r): reads its S
 //                     row with tcgen05.ld, masks (causal, window, unit range),
 //                     keeps an online softmax (a running max that is only
 //                     moved - with a rescale of its O row in TMEM - when a
-//                     tile raises it by more than 2^8), writes P as bf16 into
-//                     the swizzled shared-memory layout the second MMA reads,
-//                     and at the end normalises O and stores it.
+//                     tile raises it by more than 2^8), writes P as packed
+//                     bf16 back over the S tile it came from, and at the end
+//                     normalises O and stores it.
 //
+// Keeping P in tensor memory makes it double-buffered with S for free: the
+// softmax of tile i+1 never waits for the P.V product of tile i; the S MMA of
+// tile i+2 waits for it instead (it overwrites that buffer).
 // Every wait is bounded; a wait that gives up sets kErrTimeout and the CTA
 // drains and returns.
 #include <cuda.h>
@@ -45,19 +48,17 @@ struct TcCfg {
   static constexpr int DH = D / 64;  // 64-dim (128-byte) boxes per row
   static constexpr int kQBytes = BM * D * 2;
   static constexpr int kKVBytes = BN * D * 2;
-  static constexpr int kPBytes = BM * BN * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + KST * kKVBytes;
-  static constexpr int kOffP = kOffV + VST * kKVBytes;
-  static constexpr int kOffBar = kOffP + kPBytes;
+  static constexpr int kOffBar = kOffV + VST * kKVBytes;
   // q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST],
-  // s_full[2], s_free[2], p_full, pv_done, o_free
-  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + 2 + 2 + 3 + 2 * UnitQueue::kDepth;
+  // s_full[2], p_full[2], pv_done[2], o_free, unit queue full/empty
+  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 2 * UnitQueue::kDepth;
   static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + UnitQueue::kDepth * 4;
   static constexpr int kThreads = 192;
   static constexpr uint32_t kTmemCols = 256;
-  static constexpr uint32_t kColS = 0;     // S buffers at columns 0 and BN
+  static constexpr uint32_t kColS = 0;       // S (then P) buffers at columns 0 and BN
   static constexpr uint32_t kColO = 2 * BN;  // O at columns 2*BN .. 2*BN + D
   static_assert(kColO + D <= kTmemCols, "TMEM budget");
 };
@@ -107,6 +108,39 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 3-input maximum (sm_100): one instruction for two comparisons.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1) as one packed f32x2 FMA.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+// (d0, d1) += (a0, a1) as one packed f32x2 add.
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rd;\n\t"
+      "mov.b64 rd, {%0, %1};\n\tmov.b64 ra, {%2, %3};\n\t"
+      "add.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+// D[tmem] (+)= A[tmem] * B[smem]: A is M x K bf16 packed two per 32-bit
+// column (row m in lane m), B given by a matrix descriptor.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int32_t* err, bool& ok) {
   if (!ok) return false;
@@ -132,7 +166,6 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
   unsigned char* sQ = smem + C::kOffQ;
   unsigned char* sK = smem + C::kOffK;
   unsigned char* sV = smem + C::kOffV;
-  unsigned char* sP = smem + C::kOffP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* q_empty = q_full + 1;
@@ -141,10 +174,9 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
   uint64_t* v_full = k_empty + C::KST;
   uint64_t* v_empty = v_full + C::VST;
   uint64_t* s_full = v_empty + C::VST;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint64_t* o_free = pv_done + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* o_free = pv_done + 2;
   uint64_t* uq_full = o_free + 1;
   uint64_t* uq_empty = uq_full + UnitQueue::kDepth;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
@@ -169,10 +201,9 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&s_full[i], 1);
-      ptx::mbar_init(&s_free[i], 4);
+      ptx::mbar_init(&p_full[i], 4);
+      ptx::mbar_init(&pv_done[i], 1);
     }
-    ptx::mbar_init(p_full, 4);
-    ptx::mbar_init(pv_done, 1);
     ptx::mbar_init(o_free, 4);
     uq.init();
     ptx::fence_mbar_init();
@@ -261,23 +292,25 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
       constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(C::BM, C::BN, 0, 0);
       constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(C::BM, D, 0, 1);
       const uint32_t q_addr = ptx::smem_u32(sQ), k_addr = ptx::smem_u32(sK);
-      const uint32_t v_addr = ptx::smem_u32(sV), p_addr = ptx::smem_u32(sP);
+      const uint32_t v_addr = ptx::smem_u32(sV);
       int gt = 0, un = 0;
-      // O += P V for global tile t; `first` starts a unit's accumulation and
-      // must wait until the previous unit's epilogue has read O.
+      // O += P V for global tile t, P in the TMEM S buffer t&1 (bf16 packed,
+      // 16 keys = 8 columns per MMA step); `first` starts a unit's
+      // accumulation and must wait until the previous unit's epilogue has
+      // read O.
       auto issue_pv = [&](int t, bool first) {
-        const int vs = t % C::VST;
+        const int vs = t % C::VST, pb = t & 1;
         if (!wait_or_flag(&v_full[vs], (t / C::VST) & 1, err, ok)) return;
-        if (!wait_or_flag(p_full, t & 1, err, ok)) return;
+        if (!wait_or_flag(&p_full[pb], (t >> 1) & 1, err, ok)) return;
         if (first && un >= 1 && !wait_or_flag(o_free, (un - 1) & 1, err, ok)) return;
         ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          const uint64_t ad = ptx::smem_desc_sw128(p_addr + (kk >> 2) * C::BM * 128 + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = ptx::smem_desc_sw128(v_addr + vs * C::kKVBytes + kk * 16 * 128, C::BN * 128, 1024);
-          ptx::mma_bf16(tmem + C::kColO, ad, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + C::kColO, tmem + C::kColS + pb * C::BN + kk * 8, bd, idesc_pv,
+                      (!first || kk > 0) ? 1u : 0u);
         }
-        ptx::mma_commit(pv_done);
+        ptx::mma_commit(&pv_done[pb]);
         ptx::mma_commit(&v_empty[vs]);
       };
       for (;; ++un) {
@@ -293,7 +326,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
         for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
           const int ks = gt % C::KST, sb = gt & 1;
           if (!wait_or_flag(&k_full[ks], (gt / C::KST) & 1, err, ok)) break;
-          if (gt >= 2 && !wait_or_flag(&s_free[sb], ((gt >> 1) - 1) & 1, err, ok)) break;
+          // S buffer sb still holds P of tile gt-2 until its P.V is done
+          if (gt >= 2 && !wait_or_flag(&pv_done[sb], ((gt >> 1) - 1) & 1, err, ok)) break;
           ptx::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -336,113 +370,105 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
       for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
         const int sb = gt & 1;
         const int k0 = x.k00 + i * C::BN;
-        if (!warp_live) {
-          // padding rows: release S at once, write no P. Waiting for the
-          // previous PV keeps this warp from arriving twice in one phase.
-          if (!wait_or_flag(&s_full[sb], (gt >> 1) & 1, err, ok)) break;
-          if (lane == 0) ptx::mbar_arrive(&s_free[sb]);
-          if (gt >= 1 && !wait_or_flag(pv_done, (gt - 1) & 1, err, ok)) break;
-          if (lane == 0) ptx::mbar_arrive(p_full);
-          continue;
-        }
         if (!wait_or_flag(&s_full[sb], (gt >> 1) & 1, err, ok)) break;
-        ptx::tc_fence_after();
-        uint32_t raw[C::BN];
+        if (warp_live) {
+          ptx::tc_fence_after();
+          uint32_t raw[C::BN];
 #pragma unroll
-        for (int c = 0; c < C::BN / 32; ++c)
-          ptx::tmem_ld32(tmem + lane_base + C::kColS + sb * C::BN + c * 32,
-                         *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
-        ptx::tmem_ld_wait();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&s_free[sb]);
-        float sv[C::BN];
-        // mask and tile max
-        const int c_lo = lower - k0, c_hi = upper - k0;
-        float mt = -INFINITY;
-        if (c_lo <= 0 && c_hi >= C::BN) {
+          for (int c = 0; c < C::BN / 32; ++c)
+            ptx::tmem_ld32(tmem + lane_base + C::kColS + sb * C::BN + c * 32,
+                           *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
+          ptx::tmem_ld_wait();
+          float sv[C::BN];
+          // mask, then the tile max as a tree of 3-input maxima (8 independent
+          // chains, so the reduction is not one 64-long dependency chain)
+          const int c_lo = lower - k0, c_hi = upper - k0;
+          if (c_lo <= 0 && c_hi >= C::BN) {
 #pragma unroll
-          for (int c = 0; c < C::BN; ++c) {
-            sv[c] = __uint_as_float(raw[c]);
-            mt = fmaxf(mt, sv[c]);
+            for (int c = 0; c < C::BN; ++c) sv[c] = __uint_as_float(raw[c]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < C::BN; ++c) sv[c] = (c >= c_lo && c < c_hi) ? __uint_as_float(raw[c]) : -INFINITY;
           }
-        } else {
+          float mx[8];
 #pragma unroll
-          for (int c = 0; c < C::BN; ++c) {
-            sv[c] = (c >= c_lo && c < c_hi) ? __uint_as_float(raw[c]) : -INFINITY;
-            mt = fmaxf(mt, sv[c]);
+          for (int j = 0; j < 8; ++j) mx[j] = sv[j];
+#pragma unroll
+          for (int c = 8; c < C::BN; c += 16)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx[j] = max3(mx[j], sv[c + j], sv[c + 8 + j]);
+          const float mt = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+          const float mts = mt == -INFINITY ? -INFINITY : mt * a.scale_log2;
+          float alpha = 1.f;
+          if (mts > m_used + 8.f) {  // also true the first time a row sees a key
+            alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mts);
+            m_used = mts;
+            l *= alpha;
           }
-        }
-        const float mts = mt == -INFINITY ? -INFINITY : mt * a.scale_log2;
-        float alpha = 1.f;
-        if (mts > m_used + 8.f) {  // also true the first time a row sees a key
-          alpha = m_used == -INFINITY ? 0.f : ex2(m_used - mts);
-          m_used = mts;
-          l *= alpha;
-        }
-        // the previous PV must be done before O is rescaled and P rewritten
-        if (gt >= 1 && !wait_or_flag(pv_done, (gt - 1) & 1, err, ok)) break;
-        ptx::tc_fence_after();
-        if (i >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // O may be rescaled only once the P.V of the previous tile is done
+          if (i >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            if (!wait_or_flag(&pv_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, err, ok)) break;
+            ptx::tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            const uint32_t ta = tmem + lane_base + C::kColO + c * 32;
-            ptx::tmem_ld32(ta, o);
-            ptx::tmem_ld_wait();
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              const uint32_t ta = tmem + lane_base + C::kColO + c * 32;
+              ptx::tmem_ld32(ta, o);
+              ptx::tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            ptx::tmem_st32(ta, o);
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              ptx::tmem_st32(ta, o);
+            }
+            ptx::tmem_st_wait();
+          }
+          // P = 2^(s*scale - m_used), packed two bf16 per 32-bit word, written
+          // over the first BN/2 columns of this S buffer (lane r = row r).
+          // Masked keys are -inf and give 0; a row with no key yet has
+          // m_used = -inf, all its scores -inf, and neg_m = 0 keeps them 0.
+          float ls0[4] = {0.f, 0.f, 0.f, 0.f}, ls1[4] = {0.f, 0.f, 0.f, 0.f};
+          const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+          uint32_t pw[C::BN / 2];
+#pragma unroll
+          for (int c = 0; c < C::BN / 2; ++c) {
+            float x0, x1;
+            fma2(x0, x1, sv[2 * c], sv[2 * c + 1], a.scale_log2, a.scale_log2, neg_m, neg_m);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            add2(ls0[c & 3], ls1[c & 3], p0, p1);
+            __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+            pw[c] = *reinterpret_cast<uint32_t*>(&pr);
+          }
+          ptx::tmem_st32(tmem + lane_base + C::kColS + sb * C::BN, pw);
+          l += ((ls0[0] + ls1[0]) + (ls0[1] + ls1[1])) + ((ls0[2] + ls1[2]) + (ls0[3] + ls1[3]));
+          // keys at or past the sequence end may hold anything (unwritten
+          // slots, stale stage data): zero those V rows so 0 * garbage cannot
+          // reach O
+          if (k0 + C::BN > x.L) {
+            const int vs = gt % C::VST;
+            if (!wait_or_flag(&v_full[vs], (gt / C::VST) & 1, err, ok)) break;
+            const int z0 = max(0, x.L - k0);
+            const int per_dh = (C::BN - z0) * 8;  // 16-byte chunks per 64-dim half
+            const int nz = per_dh * C::DH;
+            const int n_live = min(C::BM, (x.R + 31) & ~31);  // threads of the live warps
+            for (int z = threadIdx.x; z < nz; z += n_live) {
+              const int dh = z / per_dh, rem = z - dh * per_dh;
+              const int row = z0 + rem / 8, chn = rem % 8;
+              *reinterpret_cast<uint4*>(sV + vs * C::kKVBytes + dh * C::BN * 128 + row * 128 + chn * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+            ptx::fence_proxy_async_smem();
           }
           ptx::tmem_st_wait();
         }
-        // P = 2^(s*scale - m_used) as bf16 into the 128-byte-swizzled layout:
-        // key c of row r sits in row r, 16-byte chunk (c/8) ^ (r%8). Masked
-        // keys are -inf and give 0; a row with no key yet has m_used = -inf,
-        // all its scores are -inf, and neg_m = 0 keeps that at 0 too.
-        float ls = 0.f;
-        const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-#pragma unroll
-        for (int ch = 0; ch < C::BN / 8; ++ch) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2(fmaf(sv[ch * 8 + 2 * e], a.scale_log2, neg_m));
-            const float p1 = ex2(fmaf(sv[ch * 8 + 2 * e + 1], a.scale_log2, neg_m));
-            ls += p0 + p1;
-            __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
-            w[e] = *reinterpret_cast<uint32_t*>(&pr);
-          }
-          const int atom = ch >> 3, cin = ch & 7;
-          unsigned char* dst = sP + atom * C::BM * 128 + r * 128 + ((cin ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        l += ls;
-        // keys at or past the sequence end may hold anything (unwritten
-        // slots, stale stage data): zero those V rows so 0 * garbage cannot
-        // reach O
-        if (k0 + C::BN > x.L) {
-          const int vs = gt % C::VST;
-          if (!wait_or_flag(&v_full[vs], (gt / C::VST) & 1, err, ok)) break;
-          const int z0 = max(0, x.L - k0);
-          const int per_dh = (C::BN - z0) * 8;  // 16-byte chunks per 64-dim half
-          const int nz = per_dh * C::DH;
-          const int n_live = min(C::BM, (x.R + 31) & ~31);  // threads of the live warps
-          for (int z = threadIdx.x; z < nz; z += n_live) {
-            const int dh = z / per_dh, rem = z - dh * per_dh;
-            const int row = z0 + rem / 8, chn = rem % 8;
-            *reinterpret_cast<uint4*>(sV + vs * C::kKVBytes + dh * C::BN * 128 + row * 128 + chn * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
-        }
-        ptx::fence_proxy_async_smem();
+        // padding warps write no P: arriving right after their s_full wait
+        // is safe, because tile gt + 2 cannot start before this phase ends
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(p_full);
+        if (lane == 0) ptx::mbar_arrive(&p_full[sb]);
       }
       if (!ok) break;
       // epilogue: wait for the unit's last PV, normalise, store, free O
-      if (!wait_or_flag(pv_done, (gt - 1) & 1, err, ok)) break;
+      const int last = gt - 1;
+      if (!wait_or_flag(&pv_done[last & 1], (last >> 1) & 1, err, ok)) break;
       ptx::tc_fence_after();
       if (warp_live) {
         const int row = x.row0 + r / g;
