@@ -117,10 +117,13 @@ struct fg_kv_cache {
   size_t bytes = 0;
   bool owned = false;
   int device = 0;
-  // rotary table [rope_npos][head_dim / 2] of (cos, sin)
+  // rotary table [rope_npos][head_dim / 2] of (cos, sin): the float-rounded
+  // values, widened to double and scaled by 2^896; within a position row,
+  // pair i = 8 g + e sits at entry e * (head_dim / 16) + g (the order the
+  // kernel's threads read it in)
   double rope_theta = 0.0;
   int32_t rope_npos = 0;
-  float2* rope = nullptr;
+  double2* rope = nullptr;
   // TMA view of the pool: 2-D (head_dim, every slot row), 64 x min(B, 64) boxes
   alignas(64) CUtensorMap tm_kv;
   int tm_kv_state = 0;  // 0 = not built, 1 = built, -1 = unavailable
@@ -201,11 +204,20 @@ static fg_status ensure_rope(fg_kv_cache* c, double theta, int32_t max_pos) {
   const int half = c->head_dim / 2;
   std::vector<float> cs((size_t)cap * half), sn((size_t)cap * half);
   build_rope_rows(theta, c->head_dim, 0, (int)cap, cs.data(), sn.data(), half);
-  std::vector<float2> tab((size_t)cap * half);
-  for (size_t i = 0; i < tab.size(); ++i) tab[i] = make_float2(cs[i], sn[i]);
-  float2* dnew = nullptr;
-  FG_CUDA(cudaMalloc(&dnew, tab.size() * sizeof(float2)));
-  cudaError_t e = cudaMemcpy(dnew, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
+  std::vector<double2> tab((size_t)cap * half);
+  // stored times 2^896 (exact): the kernel widens bf16 inputs to doubles
+  // that are 2^-896 times their value, and the two scalings cancel in
+  // every product
+  const int groups = half / 8;
+  for (int64_t p = 0; p < cap; ++p)
+    for (int i = 0; i < half; ++i) {
+      const size_t src = (size_t)p * half + i;
+      tab[(size_t)p * half + (i % 8) * groups + i / 8] =
+          make_double2(std::ldexp((double)cs[src], 896), std::ldexp((double)sn[src], 896));
+    }
+  double2* dnew = nullptr;
+  FG_CUDA(cudaMalloc(&dnew, tab.size() * sizeof(double2)));
+  cudaError_t e = cudaMemcpy(dnew, tab.data(), tab.size() * sizeof(double2), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
     cudaFree(dnew);
     return cuda_fail(e, "rotary table upload");

@@ -2,15 +2,18 @@
 // into the blocked KV cache ("DeepSpeed-FastGen — paper by Holmes et al.
 // (2024)", Key points: blocked KV cache as in PagedAttention).
 //
-// One CTA per batch row (token). Each thread rotates 8 (i, i + d/2) pairs at a
-// time with 16-byte loads of both halves and writes 16-byte stores, so every
-// global access is a full, aligned 16-byte vector; a thread issues the loads
-// of four heads before it computes and stores any of them. The rotation runs in double
-// so that it rounds exactly once: a bf16 times a float product is exact in
-// double (8 + 24 significant bits), the sum rounds once, and the double is
-// rounded straight to bf16 (ties to even) - no float intermediate that could
-// round twice.
+// Units of (token, chunk of heads) stream through a three-stage shared-memory
+// ring per CTA by bulk copy; each consumer thread rotates 8 (i, i + d/2) pairs
+// at a time from there and writes 16-byte stores. The rotation runs in double
+// so that it rounds exactly as specified: a bf16 times a float product is
+// exact in double (8 + 24 significant bits), the sum rounds once to double,
+// and the double is rounded to bf16 (ties to even) through round-to-odd, so
+// no intermediate float rounding can change the result.
+#include <algorithm>
+#include <cfloat>
+
 #include "fg_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace fg {
 namespace {
@@ -19,117 +22,250 @@ namespace {
 // force the last float bit on when the truncation dropped anything ("round
 // to odd", Boldo & Melquiond 2008): with 16 spare bits between float and bf16
 // the following float -> bf16 round-to-nearest-even then equals the direct
-// rounding of the double, subnormals included.
-__device__ __forceinline__ unsigned short f64_to_bf16_rne(double x) {
+// rounding of the double, subnormals included. Exact for every double; the
+// kernel uses it only for vectors the fast path below does not cover.
+__device__ __noinline__ unsigned short f64_to_bf16_rne_slow(double x) {
   float f = __double2float_rz(x);
   if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
+// The same round-to-odd narrowing without the double comparison: when y's
+// exponent lies in float's normal range the truncation drops exactly the low
+// 29 bits of the 52-bit significand, so the sticky bit is "those bits are not
+// all zero". Above that range the truncation gives FLT_MAX with its last bit
+// already set, which rounds to infinity as y does. Below it (float subnormal
+// or zero) more bits are dropped; `tiny` keeps the smallest magnitude
+// produced, and a vector whose minimum is below FLT_MIN takes the exact path.
+__device__ __forceinline__ float f64_to_f32_odd(double y, float& tiny) {
+  const uint32_t lo = (uint32_t)__double2loint(y);
+  const float f = __uint_as_float(__float_as_uint(__double2float_rz(y)) | (uint32_t)((lo << 3) != 0u));
+  tiny = fminf(tiny, fabsf(f));
+  return f;
+}
+
+// A bf16 pattern widened to a double whose value is 2^-896 times the bf16's
+// value, by moving its 8 exponent bits to the low end of the double's 11-bit
+// exponent field (an arithmetic shift keeps the sign on top, the mask clears
+// the three bits in between). Exact for zero, subnormal and normal patterns;
+// infinities and NaNs are screened out per vector first. The rotary table is
+// stored times 2^896, so each product x * cos is exact and unscaled.
+__device__ __forceinline__ double bf16_lo_scaled(uint32_t w) {
+  return __hiloint2double((int)(((uint32_t)((int32_t)(w << 16) >> 3)) & 0x8FFFFFFFu), 0);
+}
+__device__ __forceinline__ double bf16_hi_scaled(uint32_t w) {
+  return __hiloint2double((int)(((uint32_t)((int32_t)w >> 3)) & 0x8FFFE000u), 0);
+}
+// Bit 15 or 31 is set iff the low or high bf16 of w has an all-ones exponent.
+__device__ __forceinline__ uint32_t special_bits(uint32_t w) {
+  return ((w & 0x7F807F80u) + 0x00800080u) & 0x80008000u;
+}
 __device__ __forceinline__ double bf16_lo(uint32_t w) { return (double)__uint_as_float(w << 16); }
 __device__ __forceinline__ double bf16_hi(uint32_t w) { return (double)__uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ const __nv_bfloat16* k_in(const __nv_bfloat16* k, int t, int Hkv, int h, int D) {
-  return k + ((int64_t)t * Hkv + h) * D;
+// Rotation of one word pair (two pairs (x1, x2)) the plain way, for the
+// vectors the fast path does not cover; the table entries are times 2^896.
+__device__ __noinline__ uint2 rotate_pair_slow(uint32_t a, uint32_t b, double2 r_lo, double2 r_hi) {
+  const double x1l = bf16_lo(a), x1h = bf16_hi(a), x2l = bf16_lo(b), x2h = bf16_hi(b);
+  const double cl = r_lo.x * 0x1p-896, sl = r_lo.y * 0x1p-896;
+  const double ch = r_hi.x * 0x1p-896, sh = r_hi.y * 0x1p-896;
+  const unsigned short r1l = f64_to_bf16_rne_slow(__dsub_rn(__dmul_rn(x1l, cl), __dmul_rn(x2l, sl)));
+  const unsigned short r1h = f64_to_bf16_rne_slow(__dsub_rn(__dmul_rn(x1h, ch), __dmul_rn(x2h, sh)));
+  const unsigned short r2l = f64_to_bf16_rne_slow(__dadd_rn(__dmul_rn(x2l, cl), __dmul_rn(x1l, sl)));
+  const unsigned short r2h = f64_to_bf16_rne_slow(__dadd_rn(__dmul_rn(x2h, ch), __dmul_rn(x1h, sh)));
+  return make_uint2((uint32_t)r1l | ((uint32_t)r1h << 16), (uint32_t)r2l | ((uint32_t)r2h << 16));
 }
 
+constexpr long long kWaitLimit = 1LL << 31;
+constexpr int kChunkHeads = 32;  // heads (of q | k | v, concatenated) per unit
+constexpr int kStages = 3;
+constexpr int kCtasPerSm = 4;
+constexpr int kConsumers = 128;
+
+// What the producer tells the consumers about a unit.
+struct UnitMeta {
+  int32_t t, h0, h1, blk, slot, pad[3];
+};
+
 template <int D>
-__global__ void __launch_bounds__(128) rotary_append_kernel(CacheView cache, BatchView batch,
-                                                            const __nv_bfloat16* q,
-                                                            const __nv_bfloat16* __restrict__ k,
-                                                            const __nv_bfloat16* __restrict__ v,
-                                                            __nv_bfloat16* q_rot,
-                                                            const float2* __restrict__ rope,
-                                                            int Hq) {
-  constexpr int HALF = D / 2;
+struct RotCfg {
+  static constexpr int ROW = D * 2;  // bytes per head row
+  static constexpr int HALF = D / 2;
+  static constexpr int kRows = 0;
+  static constexpr int kRope = kRows + kChunkHeads * ROW;  // HALF (cos, sin) pairs of double
+  static constexpr int kMeta = kRope + HALF * 16;
+  static constexpr int kStage = kMeta + (int)sizeof(UnitMeta);
+  static constexpr int kBar = kStages * kStage;
+  static constexpr int kSmem = kBar + 2 * kStages * 8;
+};
+
+// A unit is (token, chunk of 32 heads of the concatenated q | k | v rows).
+// Warp 4 (one lane) is the producer: for each of the CTA's units (blockIdx.x,
+// + gridDim.x, ...) it resolves the token's sequence, position and cache
+// block, writes them into the stage, and pulls the unit's rows (each of q, k
+// and v a contiguous run of whole heads) and the position's rotary row with
+// 1-D bulk copies on the stage's mbarrier. Warps 0-3 rotate from shared
+// memory and store 16-byte vectors, then free the stage. With three stages
+// the producer's dependent metadata loads and the copies stay ahead of the
+// arithmetic.
+template <int D>
+__global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_kernel(
+    CacheView cache, BatchView batch, const __nv_bfloat16* q, const __nv_bfloat16* k,
+    const __nv_bfloat16* v, __nv_bfloat16* q_rot, const double2* __restrict__ rope, int Hq, int chunks) {
+  using C = RotCfg<D>;
+  constexpr int HALF = C::HALF;
   constexpr int GROUPS = HALF / 8;  // 8-pair groups per head
-  const int t = blockIdx.x;
+  constexpr int ROW = C::ROW;
+  static_assert(kConsumers % GROUPS == 0, "consumer count must be a multiple of the groups per head");
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  uint64_t* empty = full + kStages;
   const int Hkv = cache.n_kv_heads;
-  const int s = batch.tok_seq[t];
-  const int p = batch.ctx[s] + (t - batch.cu_q[s]);
-  const int lb = p / cache.block_size;
-  const int slot = p - lb * cache.block_size;
-  int32_t blk = batch.bt[batch.bt_off[s] + lb];
-  const bool blk_ok = blk >= 0 && blk < cache.n_blocks;
-  if (!blk_ok && threadIdx.x == 0) atomicOr(batch.err, kErrBadBlock);
-  // Every thread handles the same 8-pair group i0 of several heads (the block
-  // size is a multiple of the groups per head), so its 8 (cos, sin) pairs are
-  // loaded once; all loads of a batch of heads are issued before any store.
-  static_assert(128 % GROUPS == 0, "block size must be a multiple of the groups per head");
-  const int i0 = (threadIdx.x % GROUPS) * 8;
-  float cs[8], sn[8];
-  {
-    const float4* r4 = reinterpret_cast<const float4*>(rope + (int64_t)p * HALF + i0);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float4 r = r4[e];
-      cs[2 * e] = r.x; sn[2 * e] = r.y; cs[2 * e + 1] = r.z; sn[2 * e + 1] = r.w;
+  const int n_units = batch.n_tokens * chunks;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], kConsumers / 32);
     }
+    ptx::fence_mbar_init();
   }
-  constexpr int BATCH = 4;
-  const int total = (Hq + Hkv) * GROUPS;
-  for (int base = threadIdx.x; base < total; base += BATCH * 128) {
-    uint4 a[BATCH], b[BATCH];
-#pragma unroll
-    for (int j = 0; j < BATCH; ++j) {
-      const int gi = base + j * 128;
-      if (gi >= total) break;
-      const int h = gi / GROUPS;
-      const __nv_bfloat16* src = h < Hq ? q + ((int64_t)t * Hq + h) * D
-                                        : k_in(k, t, Hkv, h - Hq, D);
-      a[j] = *reinterpret_cast<const uint4*>(src + i0);
-      b[j] = *reinterpret_cast<const uint4*>(src + HALF + i0);
-    }
-#pragma unroll
-    for (int j = 0; j < BATCH; ++j) {
-      const int gi = base + j * 128;
-      if (gi >= total) break;
-      const int h = gi / GROUPS;
-      const uint32_t aw[4] = {a[j].x, a[j].y, a[j].z, a[j].w};
-      const uint32_t bw[4] = {b[j].x, b[j].y, b[j].z, b[j].w};
-      uint32_t y1[4], y2[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const double x1l = bf16_lo(aw[e]), x1h = bf16_hi(aw[e]);
-        const double x2l = bf16_lo(bw[e]), x2h = bf16_hi(bw[e]);
-        const double cl = cs[2 * e], sl = sn[2 * e], ch = cs[2 * e + 1], sh = sn[2 * e + 1];
-        const unsigned short r1l = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1l, cl), __dmul_rn(x2l, sl)));
-        const unsigned short r1h = f64_to_bf16_rne(__dsub_rn(__dmul_rn(x1h, ch), __dmul_rn(x2h, sh)));
-        const unsigned short r2l = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2l, cl), __dmul_rn(x1l, sl)));
-        const unsigned short r2h = f64_to_bf16_rne(__dadd_rn(__dmul_rn(x2h, ch), __dmul_rn(x1h, sh)));
-        y1[e] = (uint32_t)r1l | ((uint32_t)r1h << 16);
-        y2[e] = (uint32_t)r2l | ((uint32_t)r2h << 16);
+  __syncthreads();
+
+  if (threadIdx.x >= kConsumers) {
+    // ------------------------------------------------------------ producer
+    if (threadIdx.x != kConsumers) return;
+    int it = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
+      const int st = it % kStages;
+      if (it >= kStages && !ptx::mbar_wait_bounded(&empty[st], ((it / kStages) - 1) & 1, kWaitLimit)) {
+        atomicOr(batch.err, kErrTimeout);
+        return;  // the consumers give up on the full barrier of this stage
       }
-      __nv_bfloat16* dst;
-      if (h < Hq) {
-        dst = q_rot + ((int64_t)t * Hq + h) * D;
-      } else {
-        if (!blk_ok) continue;
-        dst = cache.base + cache_offset(cache, blk, 0, h - Hq, slot);
-      }
-      *reinterpret_cast<uint4*>(dst + i0) = make_uint4(y1[0], y1[1], y1[2], y1[3]);
-      *reinterpret_cast<uint4*>(dst + HALF + i0) = make_uint4(y2[0], y2[1], y2[2], y2[3]);
+      unsigned char* stage = smem + st * C::kStage;
+      const int t = u / chunks;
+      const int h0 = (u - t * chunks) * kChunkHeads;
+      const int h1 = min(h0 + kChunkHeads, Hq + 2 * Hkv);
+      const int s = batch.tok_seq[t];
+      const int pos = batch.ctx[s] + (t - batch.cu_q[s]);
+      const int lb = pos / cache.block_size;
+      UnitMeta m;
+      m.t = t;
+      m.h0 = h0;
+      m.h1 = h1;
+      m.blk = batch.bt[batch.bt_off[s] + lb];
+      m.slot = pos - lb * cache.block_size;
+      *reinterpret_cast<UnitMeta*>(stage + C::kMeta) = m;
+      const bool rot = h0 < Hq + Hkv;
+      ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((h1 - h0) * ROW + (rot ? HALF * 16 : 0)));
+      if (rot) ptx::bulk_g2s(stage + C::kRope, rope + (int64_t)pos * HALF, HALF * 16, &full[st]);
+      // [h0, h1) cut by the q, k and v ranges of the concatenated head list
+      const int qa = h0, qb = min(h1, Hq);
+      if (qa < qb)
+        ptx::bulk_g2s(stage, q + ((int64_t)t * Hq + qa) * D, (uint32_t)((qb - qa) * ROW), &full[st]);
+      const int ka = max(h0, Hq), kb = min(h1, Hq + Hkv);
+      if (ka < kb)
+        ptx::bulk_g2s(stage + (ka - h0) * ROW, k + ((int64_t)t * Hkv + (ka - Hq)) * D,
+                      (uint32_t)((kb - ka) * ROW), &full[st]);
+      const int va = max(h0, Hq + Hkv), vb = h1;
+      if (va < vb)
+        ptx::bulk_g2s(stage + (va - h0) * ROW, v + ((int64_t)t * Hkv + (va - Hq - Hkv)) * D,
+                      (uint32_t)((vb - va) * ROW), &full[st]);
     }
+    return;
   }
-  if (!blk_ok) return;
-  constexpr int VCH = D / 8;
-  const int nv = Hkv * VCH;
-  for (int base = threadIdx.x; base < nv; base += BATCH * 128) {
-    uint4 x[BATCH];
-#pragma unroll
-    for (int j = 0; j < BATCH; ++j) {
-      const int ci = base + j * 128;
-      if (ci >= nv) break;
-      const int h = ci / VCH;
-      x[j] = *reinterpret_cast<const uint4*>(v + ((int64_t)t * Hkv + h) * D + (ci - h * VCH) * 8);
+
+  // -------------------------------------------------------------- consumers
+  const int g = threadIdx.x % GROUPS;  // this thread's 8-pair group of every head it rotates
+  const int i0 = g * 8;
+  int it = 0;
+  for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
+    const int st = it % kStages;
+    // the whole warp learns together whether the stage arrived
+    const bool landed = ptx::mbar_wait_bounded(&full[st], (it / kStages) & 1, kWaitLimit);
+    if (!__all_sync(0xffffffffu, landed)) {
+      if ((threadIdx.x & 31) == 0) atomicOr(batch.err, kErrTimeout);
+      return;
     }
+    const unsigned char* stage = smem + st * C::kStage;
+    const UnitMeta m = *reinterpret_cast<const UnitMeta*>(stage + C::kMeta);
+    const bool blk_ok = m.blk >= 0 && m.blk < cache.n_blocks;
+    if (!blk_ok && threadIdx.x == 0) atomicOr(batch.err, kErrBadBlock);
+    const int n_rot = max(0, min(m.h1, Hq + Hkv) - m.h0);  // rotated heads in this unit
+    if (n_rot > 0) {
+      // the rotary row is stored pair 8 g + e at entry e * GROUPS + g, so
+      // these loads are conflict-free
+      const double2* rs = reinterpret_cast<const double2*>(stage + C::kRope);
+      double cs[8], sn[8];
 #pragma unroll
-    for (int j = 0; j < BATCH; ++j) {
-      const int ci = base + j * 128;
-      if (ci >= nv) break;
-      const int h = ci / VCH;
-      *reinterpret_cast<uint4*>(cache.base + cache_offset(cache, blk, 1, h, slot) + (ci - h * VCH) * 8) = x[j];
+      for (int e = 0; e < 8; ++e) {
+        const double2 r = rs[e * GROUPS + g];
+        cs[e] = r.x;
+        sn[e] = r.y;
+      }
+      for (int hl = threadIdx.x / GROUPS; hl < n_rot; hl += kConsumers / GROUPS) {
+        const int h = m.h0 + hl;
+        const uint4 a = *reinterpret_cast<const uint4*>(stage + hl * ROW + i0 * 2);
+        const uint4 b = *reinterpret_cast<const uint4*>(stage + hl * ROW + (HALF + i0) * 2);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+        uint32_t y1[4], y2[4];
+        uint32_t special = 0;
+        float tiny = FLT_MAX;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          special |= special_bits(aw[e]) | special_bits(bw[e]);
+          const double x1l = bf16_lo_scaled(aw[e]), x1h = bf16_hi_scaled(aw[e]);
+          const double x2l = bf16_lo_scaled(bw[e]), x2h = bf16_hi_scaled(bw[e]);
+          const double cl = cs[2 * e], sl = sn[2 * e], ch = cs[2 * e + 1], sh = sn[2 * e + 1];
+          // both products are exact, so one fused multiply-add rounds the
+          // difference exactly once
+          const double r1l = __fma_rn(x1l, cl, -__dmul_rn(x2l, sl));
+          const double r1h = __fma_rn(x1h, ch, -__dmul_rn(x2h, sh));
+          const double r2l = __fma_rn(x2l, cl, __dmul_rn(x1l, sl));
+          const double r2h = __fma_rn(x2h, ch, __dmul_rn(x1h, sh));
+          __nv_bfloat162 p1 =
+              __floats2bfloat162_rn(f64_to_f32_odd(r1l, tiny), f64_to_f32_odd(r1h, tiny));
+          __nv_bfloat162 p2 =
+              __floats2bfloat162_rn(f64_to_f32_odd(r2l, tiny), f64_to_f32_odd(r2h, tiny));
+          y1[e] = *reinterpret_cast<uint32_t*>(&p1);
+          y2[e] = *reinterpret_cast<uint32_t*>(&p2);
+        }
+        if (special != 0u || tiny < FLT_MIN) {
+          // an infinite or NaN input, or a result below float's normal
+          // range: redo the vector with plain widening and the exact narrowing
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint2 r = rotate_pair_slow(aw[e], bw[e], rs[(2 * e) * GROUPS + g], rs[(2 * e + 1) * GROUPS + g]);
+            y1[e] = r.x;
+            y2[e] = r.y;
+          }
+        }
+        __nv_bfloat16* dst;
+        if (h < Hq) {
+          dst = q_rot + ((int64_t)m.t * Hq + h) * D;
+        } else {
+          if (!blk_ok) continue;
+          dst = cache.base + cache_offset(cache, m.blk, 0, h - Hq, m.slot);
+        }
+        *reinterpret_cast<uint4*>(dst + i0) = make_uint4(y1[0], y1[1], y1[2], y1[3]);
+        *reinterpret_cast<uint4*>(dst + HALF + i0) = make_uint4(y2[0], y2[1], y2[2], y2[3]);
+      }
     }
+    if (blk_ok) {
+      // V heads of the unit: a plain copy into the cache slots
+      constexpr int VCH = D / 8;  // 16-byte pieces per head
+      const int v0 = max(m.h0, Hq + Hkv);
+      const int nv = max(0, m.h1 - v0) * VCH;
+      for (int ci = threadIdx.x; ci < nv; ci += kConsumers) {
+        const int hl = ci / VCH, c = ci - hl * VCH;
+        const int h = v0 + hl - Hq - Hkv;
+        *reinterpret_cast<uint4*>(cache.base + cache_offset(cache, m.blk, 1, h, m.slot) + c * 8) =
+            *reinterpret_cast<const uint4*>(stage + (v0 - m.h0 + hl) * ROW + c * 16);
+      }
+    }
+    // this warp is done with the stage
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(&empty[st]);
   }
 }
 
@@ -137,14 +273,22 @@ __global__ void __launch_bounds__(128) rotary_append_kernel(CacheView cache, Bat
 
 cudaError_t launch_rotary_append(const CacheView& cache, const BatchView& batch,
                                  const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                 const __nv_bfloat16* v, __nv_bfloat16* q_rot, const float2* rope,
+                                 const __nv_bfloat16* v, __nv_bfloat16* q_rot, const double2* rope,
                                  int n_q_heads, cudaStream_t stream) {
   if (batch.n_tokens == 0) return cudaSuccess;
-  dim3 grid(batch.n_tokens), block(128);
+  const int chunks = (n_q_heads + 2 * cache.n_kv_heads + kChunkHeads - 1) / kChunkHeads;
+  const int64_t units = (int64_t)batch.n_tokens * chunks;
+  if (units > (int64_t)1 << 30) return cudaErrorInvalidConfiguration;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 148;
+  const int grid = (int)std::min<int64_t>(units, (int64_t)sms * kCtasPerSm);
   if (cache.head_dim == 128)
-    rotary_append_kernel<128><<<grid, block, 0, stream>>>(cache, batch, q, k, v, q_rot, rope, n_q_heads);
+    rotary_append_kernel<128><<<grid, kConsumers + 32, RotCfg<128>::kSmem, stream>>>(
+        cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
   else
-    rotary_append_kernel<64><<<grid, block, 0, stream>>>(cache, batch, q, k, v, q_rot, rope, n_q_heads);
+    rotary_append_kernel<64><<<grid, kConsumers + 32, RotCfg<64>::kSmem, stream>>>(
+        cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
   return cudaGetLastError();
 }
 
