@@ -231,6 +231,14 @@ fg_status fg_ragged_batch_set_overlap(fg_ragged_batch* batch, int32_t enable);
  * its buffers (the access was skipped), or FG_ERR_TIMEOUT. */
 fg_status fg_device_status(fg_ragged_batch* batch, void* stream);
 
+/* Self-test of the bounded waits the kernels use instead of unbounded spins:
+ * launches one CTA that waits, with a limit of `limit_cycles` SM clocks, on
+ * an mbarrier nothing will ever complete, then reads the status the CTA
+ * wrote. Returns FG_ERR_TIMEOUT when the wait gave up as designed (the
+ * expected result), FG_ERR_DEVICE_CHECK if it did not, FG_ERR_CUDA on a
+ * runtime error. Synchronises `stream`. No device fault is involved. */
+fg_status fg_selftest_bounded_wait(int64_t limit_cycles, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Host-only helpers                                                          */
 /* ------------------------------------------------------------------------ */

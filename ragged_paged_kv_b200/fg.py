@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
         "fg_ragged_batch_set_timing": [V, I32],
         "fg_ragged_batch_set_overlap": [V, I32],
         "fg_host_profile_us": [V, ctypes.POINTER(ctypes.c_double), I32],
+        "fg_selftest_bounded_wait": [I64, V],
         "fg_attention_kernel_ms": [V, _c_float_p],
         "fg_rotary_table": [D, I32, I32, I32, _c_float_p, _c_float_p],
     }
