@@ -6,8 +6,8 @@ One step = one Dynamic SplitFuse forward pass of the attention path over the
 Llama-2-7B-shape SplitFuse snapshot (32/32 heads, d=128, block 64, budget
 2048 = 31 decodes + one 2017-token prompt chunk): batch put (metadata upload),
 rotary + paged append, ragged attention (+ split-KV combine). Inputs are
-resident in HBM when timing starts; L2 is flushed (256 MB write) between
-steps, outside the timed events. Prints one JSON line (rank 0).
+resident in HBM when timing starts; L2 is flushed (256 MB written, then read
+back) between steps, outside the timed events. Prints one JSON line (rank 0).
 
 With N > 1 (torchrun) every rank runs its own replica of the step on its own
 GPU (the path has no exchange step, so no collective is on the data path);
@@ -280,6 +280,7 @@ def run_fg(args, w, rank, ws, local_rank):
         t0 = time.perf_counter()
         batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, stream)
         t1 = time.perf_counter()
+        ev[3].record(stream)
         fg.rotary_kv_append(cache, batch, q, k, v, q_rot, w.n_q_heads, w.rope_theta, stream)
         t2 = time.perf_counter()
         ev[1].record(stream)
@@ -292,10 +293,14 @@ def run_fg(args, w, rank, ws, local_rank):
         host_parts["attention"] += t3 - t2
 
     def flush_l2():
+        # write a buffer larger than L2 (evicts every line of the step), then
+        # read it back, so that the write-back of the dirty flush lines is
+        # paid here and not by the first kernel of the next step
         with torch.cuda.stream(stream):
             flush.zero_()
+            flush.sum()
 
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     for _ in range(args.warmup):
         step(mk())
         flush_l2()
@@ -303,23 +308,27 @@ def run_fg(args, w, rank, ws, local_rank):
     batch.device_status(stream)
 
     evs = [mk() for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
     host_s = 0.0
     for k_ in host_parts:
         host_parts[k_] = 0.0
     batch.host_profile_us(reset=True)
+    # the sampler thread is started before the barrier, and every step
+    # (the first included) is preceded by the L2 flush, so the device has
+    # queued work while the host enqueues a step, as it does between steps
     with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize()
         for i in range(args.steps):
+            flush_l2()
             t0 = time.perf_counter()
             step(evs[i])
             host_s += time.perf_counter() - t0
-            flush_l2()
         torch.cuda.synchronize()
-    barrier()
+        barrier()
     lib_host = {k_: v_ / args.steps for k_, v_ in batch.host_profile_us(reset=True).items()}
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
-    put_append_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / len(evs)
+    put_ms = sum(e[0].elapsed_time(e[3]) for e in evs) / len(evs)
+    append_ms = sum(e[3].elapsed_time(e[1]) for e in evs) / len(evs)
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
     ms_local = sum(step_ms) / len(step_ms)
     ms = max_over_ranks(ms_local, dev)
@@ -394,7 +403,8 @@ def run_fg(args, w, rank, ws, local_rank):
     roof.update({"peak_source": f"{src} (MEASURED_PEAKS.json)" if src == "measured" else src,
                  "kernel_ms": kernel_ms,
                  "attention_call_ms": attn_ms_mean,
-                 "put_append_ms": put_append_ms,
+                 "put_ms": put_ms,
+                 "append_ms": append_ms,
                  "host_enqueue_ms_per_step": 1000 * host_s / args.steps,
                  "host_ms_per_call": {k_: 1000 * v_ / args.steps for k_, v_ in host_parts.items()},
                  "library_host_us_per_step": lib_host,
@@ -410,7 +420,7 @@ def run_fg(args, w, rank, ws, local_rank):
         "config": {"workload": f"{w.name} ({w.n_q_heads}/{w.n_kv_heads} heads, d={w.head_dim})", "tokens_per_gpu": w.n_tokens,
                    "seqs": w.n_seqs, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
                    "head_dim": w.head_dim, "block_size": w.block_size, "pool_blocks": w.n_blocks,
-                   "note": w.note, "l2": "flushed between steps (256 MB write, outside the events)",
+                   "note": w.note, "l2": "flushed between steps (256 MB write, then the same 256 MB read back; outside the events)",
                    "parallelism": f"replicas x{ws}"},
         "roofline": roof,
         "e2e": {"value": tokens / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
