@@ -24,8 +24,9 @@
 //                     normalises O and stores it.
 //
 // Keeping P in tensor memory makes it double-buffered with S for free: the
-// softmax of tile i+1 never waits for the P.V product of tile i; the S MMA of
-// tile i+2 waits for it instead (it overwrites that buffer).
+// softmax of tile i+1 never waits for the P.V product of tile i, and the S
+// product of tile i+2, which overwrites that buffer, is issued right behind
+// that P.V (the tensor core runs one thread's MMAs in issue order).
 // Every wait is bounded; a wait that gives up sets kErrTimeout and the CTA
 // drains and returns.
 #include <cuda.h>
@@ -113,23 +114,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float m;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
   return m;
-}
-// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1) as one packed f32x2 FMA.
-__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
-                                     float c1) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-// (d0, d1) += (a0, a1) as one packed f32x2 add.
-__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
-  asm("{\n\t.reg .b64 ra, rd;\n\t"
-      "mov.b64 rd, {%0, %1};\n\tmov.b64 ra, {%2, %3};\n\t"
-      "add.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(d0), "+f"(d1)
-      : "f"(a0), "f"(a1));
 }
 // D[tmem] (+)= A[tmem] * B[smem]: A is M x K bf16 packed two per 32-bit
 // column (row m in lane m), B given by a matrix descriptor.
@@ -326,8 +310,10 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
         for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
           const int ks = gt % C::KST, sb = gt & 1;
           if (!wait_or_flag(&k_full[ks], (gt / C::KST) & 1, err, ok)) break;
-          // S buffer sb still holds P of tile gt-2 until its P.V is done
-          if (gt >= 2 && !wait_or_flag(&pv_done[sb], ((gt >> 1) - 1) & 1, err, ok)) break;
+          // S buffer sb holds P of tile gt-2, which the P.V product issued
+          // just before this one reads: tcgen05.mma operations issued by one
+          // thread execute in issue order, so this S product is queued
+          // behind that P.V instead of waiting for its completion here
           ptx::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -383,18 +369,20 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
           // mask, then the tile max as a tree of 3-input maxima (8 independent
           // chains, so the reduction is not one 64-long dependency chain)
           const int c_lo = lower - k0, c_hi = upper - k0;
-          if (c_lo <= 0 && c_hi >= C::BN) {
 #pragma unroll
-            for (int c = 0; c < C::BN; ++c) sv[c] = __uint_as_float(raw[c]);
-          } else {
+          for (int c = 0; c < C::BN; ++c) sv[c] = __uint_as_float(raw[c]);
+          // most tiles need no mask; the test is a warp vote, so the selects
+          // below run (for the whole warp) only on tiles that need them
+          if (__any_sync(0xffffffffu, c_lo > 0 || c_hi < C::BN)) {
 #pragma unroll
-            for (int c = 0; c < C::BN; ++c) sv[c] = (c >= c_lo && c < c_hi) ? __uint_as_float(raw[c]) : -INFINITY;
+            for (int c = 0; c < C::BN; ++c)
+              if (c < c_lo || c >= c_hi) sv[c] = -INFINITY;
           }
           float mx[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) mx[j] = sv[j];
+          for (int j = 0; j < 8; ++j) mx[j] = fmaxf(sv[j], sv[8 + j]);
 #pragma unroll
-          for (int c = 8; c < C::BN; c += 16)
+          for (int c = 16; c < C::BN; c += 16)
 #pragma unroll
             for (int j = 0; j < 8; ++j) mx[j] = max3(mx[j], sv[c + j], sv[c + 8 + j]);
           const float mt = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
@@ -415,8 +403,13 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
               const uint32_t ta = tmem + lane_base + C::kColO + c * 32;
               ptx::tmem_ld32(ta, o);
               ptx::tmem_ld_wait();
+              const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              for (int e = 0; e < 32; e += 2) {
+                const float2 r = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), al2);
+                o[e] = __float_as_uint(r.x);
+                o[e + 1] = __float_as_uint(r.y);
+              }
               ptx::tmem_st32(ta, o);
             }
             ptx::tmem_st_wait();
@@ -425,20 +418,24 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
           // over the first BN/2 columns of this S buffer (lane r = row r).
           // Masked keys are -inf and give 0; a row with no key yet has
           // m_used = -inf, all its scores -inf, and neg_m = 0 keeps them 0.
-          float ls0[4] = {0.f, 0.f, 0.f, 0.f}, ls1[4] = {0.f, 0.f, 0.f, 0.f};
+          // the scale-and-shift and the running sums use the packed f32x2
+          // FMA/add, two keys per instruction
+          float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
           const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+          const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(neg_m, neg_m);
           uint32_t pw[C::BN / 2];
 #pragma unroll
           for (int c = 0; c < C::BN / 2; ++c) {
-            float x0, x1;
-            fma2(x0, x1, sv[2 * c], sv[2 * c + 1], a.scale_log2, a.scale_log2, neg_m, neg_m);
-            const float p0 = ex2(x0), p1 = ex2(x1);
-            add2(ls0[c & 3], ls1[c & 3], p0, p1);
-            __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+            const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
+            const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+            ls[c & 3] = __fadd2_rn(ls[c & 3], pp);
+            __nv_bfloat162 pr = __floats2bfloat162_rn(pp.x, pp.y);
             pw[c] = *reinterpret_cast<uint32_t*>(&pr);
           }
           ptx::tmem_st32(tmem + lane_base + C::kColS + sb * C::BN, pw);
-          l += ((ls0[0] + ls1[0]) + (ls0[1] + ls1[1])) + ((ls0[2] + ls1[2]) + (ls0[3] + ls1[3]));
+          const float2 l01 = __fadd2_rn(ls[0], ls[1]), l23 = __fadd2_rn(ls[2], ls[3]);
+          l += (l01.x + l01.y) + (l23.x + l23.y);
           // keys at or past the sequence end may hold anything (unwritten
           // slots, stale stage data): zero those V rows so 0 * garbage cannot
           // reach O
