@@ -70,6 +70,12 @@ struct DtcArgs {
   float scale_log2;
   int n_items;
   int* counter;  // next-unit counter, zero at launch
+  // When the query-tile kernel runs beside this one on SMs [0, sm_tc_end):
+  // a CTA placed there while query tiles are still unclaimed leaves at once
+  // (the SM belongs to that kernel); one placed there later helps here.
+  int sm_tc_end;
+  const int* tc_counter;
+  int n_tc;
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -113,6 +119,7 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
   using C = DtcCfg;
   constexpr int D = C::D;
   extern __shared__ __align__(1024) unsigned char smem[];
+  if (ptx::sm_id() < a.sm_tc_end && *(volatile const int*)a.tc_counter < a.n_tc) return;
   if (ptx::smem_u32(smem) & 1023u) {
     if (threadIdx.x == 0) atomicOr(a.batch.err, kErrBadIndex);
     return;
@@ -448,6 +455,11 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
+  // Launched behind the query-tile kernel (programmatic dependent launch),
+  // this grid may start before that one ends; it does not read its results,
+  // but a grid launched behind this one (the combine) must be able to rely
+  // on both: so no CTA ends before the preceding grid has.
+  ptx::grid_dependency_wait();
 }
 
 }  // namespace
@@ -456,6 +468,7 @@ cudaError_t launch_attention_decode_tc(const void* tm_q1, const void* tm_kv, con
                                        const BatchView& batch, const WorkItem* items, int n_items,
                                        __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
                                        int g, float scale_log2, int grid, int* counter,
+                                       int sm_tc_end, const int* tc_counter, int n_tc, bool pdl,
                                        cudaStream_t stream) {
   if (n_items == 0) return cudaSuccess;
   static bool configured = false;
@@ -470,11 +483,21 @@ cudaError_t launch_attention_decode_tc(const void* tm_q1, const void* tm_kv, con
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  DtcArgs args{cache, batch, items, out, part_o, part_ml, n_q_heads, g, scale_log2, n_items, counter};
+  DtcArgs args{cache, batch, items, out, part_o, part_ml, n_q_heads, g, scale_log2, n_items, counter,
+               sm_tc_end, tc_counter, n_tc};
   grid = grid < 1 ? 1 : (grid > n_items ? n_items : grid);
-  attn_decode_tc_kernel<<<grid, DtcCfg::kThreads, DtcCfg::kSmem, stream>>>(
-      *static_cast<const CUtensorMap*>(tm_q1), *static_cast<const CUtensorMap*>(tm_kv), args);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(DtcCfg::kThreads);
+  cfg.dynamicSmemBytes = DtcCfg::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_decode_tc_kernel, *static_cast<const CUtensorMap*>(tm_q1),
+                            *static_cast<const CUtensorMap*>(tm_kv), args);
 }
 
 }  // namespace fg

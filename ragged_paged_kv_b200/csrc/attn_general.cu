@@ -9,6 +9,7 @@
 #include <cfloat>
 
 #include "fg_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace fg {
 namespace {
@@ -185,25 +186,33 @@ __global__ void __launch_bounds__(128) combine_kernel(BatchView batch,
                                                       const float* __restrict__ part_ml,
                                                       __nv_bfloat16* __restrict__ out, int Hq,
                                                       int g) {
+  // launched behind the kernel that wrote the partials: wait for it (and
+  // everything before it) to finish before reading them
+  ptx::grid_dependency_wait();
   const CombineItem it = items[blockIdx.x];
-  const int r = blockIdx.y * 4 + (threadIdx.x >> 5);
+  const int r = blockIdx.y * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= it.n_rows) return;
-  float M = -INFINITY;
-  for (int i = 0; i < it.n_splits; ++i)
-    M = fmaxf(M, part_ml[(int64_t)(it.part_base + i * it.n_rows + r) * 2]);
+  // one pass of running log-sum-exp merges; four splits' loads in flight at once
   constexpr int PER = D / 32;
-  float o[PER];
+  float M = -INFINITY, L = 0.f, o[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) o[e] = 0.f;
-  float L = 0.f;
+#pragma unroll 4
   for (int i = 0; i < it.n_splits; ++i) {
     const int64_t pr = it.part_base + (int64_t)i * it.n_rows + r;
-    const float m = part_ml[pr * 2];
-    const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
-    L = fmaf(w, part_ml[pr * 2 + 1], L);
+    const float m = part_ml[pr * 2], l = part_ml[pr * 2 + 1];
+    float x[PER];
 #pragma unroll
-    for (int e = 0; e < PER; ++e) o[e] = fmaf(w, part_o[pr * D + lane + 32 * e], o[e]);
+    for (int e = 0; e < PER; ++e) x[e] = part_o[pr * D + lane + 32 * e];
+    if (m != -INFINITY) {
+      const float Mn = fmaxf(M, m);
+      const float s_old = M == -INFINITY ? 0.f : exp2f(M - Mn), s_new = exp2f(m - Mn);
+      L = fmaf(L, s_old, l * s_new);
+#pragma unroll
+      for (int e = 0; e < PER; ++e) o[e] = fmaf(o[e], s_old, x[e] * s_new);
+      M = Mn;
+    }
   }
   const int j = r / g, h = it.kv_head * g + (r - j * g);
   const int64_t row = batch.cu_q[it.seq] + it.tok_begin + j;
@@ -232,15 +241,23 @@ cudaError_t launch_attention_general(const CacheView& cache, const BatchView& ba
 
 cudaError_t launch_combine(const BatchView& batch, const CombineItem* items, int n_items,
                            int max_rows, const float* part_o, const float* part_ml,
-                           __nv_bfloat16* out, int n_q_heads, int g, int head_dim,
+                           __nv_bfloat16* out, int n_q_heads, int g, int head_dim, bool pdl,
                            cudaStream_t stream) {
   if (n_items == 0) return cudaSuccess;
-  dim3 grid(n_items, (max_rows + 3) / 4);
+  // one warp per row, up to four rows per CTA
+  const int warps = max_rows < 4 ? (max_rows < 1 ? 1 : max_rows) : 4;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_items, (max_rows + warps - 1) / warps);
+  cfg.blockDim = dim3(32 * warps);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
   if (head_dim == 128)
-    combine_kernel<128><<<grid, 128, 0, stream>>>(batch, items, part_o, part_ml, out, n_q_heads, g);
-  else
-    combine_kernel<64><<<grid, 128, 0, stream>>>(batch, items, part_o, part_ml, out, n_q_heads, g);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, combine_kernel<128>, batch, items, part_o, part_ml, out, n_q_heads, g);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<64>, batch, items, part_o, part_ml, out, n_q_heads, g);
 }
 
 }  // namespace fg

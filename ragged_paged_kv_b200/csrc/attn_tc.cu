@@ -77,6 +77,7 @@ struct TcArgs {
   int window;
   int n_items;
   int* counter;  // next-unit counter, zero at launch
+  int sm_end;    // only CTAs on SMs with id < sm_end take units (the others leave at once)
 };
 
 // What every role needs to know about one unit.
@@ -142,6 +143,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
   using C = TcCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = smem_raw;
+  // SMs outside the kernel's share are left to the decode kernel
+  if (ptx::sm_id() >= a.sm_end) return;
   // the swizzled tiles need 1024-byte alignment of the dynamic window
   if (ptx::smem_u32(smem_raw) & 1023u) {
     if (threadIdx.x == 0) atomicOr(a.batch.err, kErrBadIndex);
@@ -263,6 +266,9 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
           }
         }
       }
+      // every unit is claimed: a grid launched behind this one (the decode
+      // kernel) may take SMs as this kernel's CTAs leave
+      ptx::allow_dependent_launch();
       // let in-flight loads land before the CTA can exit
       for (int t = max(0, gt - C::KST); t < gt && ok; ++t)
         wait_or_flag(&k_full[t % C::KST], (t / C::KST) & 1, err, ok);
@@ -516,31 +522,23 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
   }
 }
 
-// Dynamic shared memory requested when the kernel must leave each SM to one
-// CTA of its own beside one decode CTA: two CTAs of this size (plus the 1 KB
-// each CTA reserves) exceed an SM's 228 KB, one of them plus a decode CTA
-// does not.
-constexpr int kTcSmemExclusive = 117760;
-
 template <int D>
-cudaError_t launch_tc_d(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const TcArgs& args,
-                        int grid, bool exclusive, cudaStream_t stream) {
+cudaError_t launch_tc_d(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const TcArgs& args, int grid,
+                        cudaStream_t stream) {
   using C = TcCfg<D>;
-  static_assert(C::kSmem <= kTcSmemExclusive, "padding below the kernel's own need");
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kTcSmemExclusive);
+    cudaError_t e =
+        cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
-    // the largest shared-memory carveout, so CTAs of different kernels can
-    // share an SM
+    // the largest shared-memory carveout: two CTAs per SM, and a decode CTA
+    // beside one when the kernels share the GPU
     e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  attn_tc_kernel<D><<<grid, C::kThreads, exclusive ? kTcSmemExclusive : C::kSmem, stream>>>(tm_q, tm_kv,
-                                                                                          args);
+  attn_tc_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tm_q, tm_kv, args);
   return cudaGetLastError();
 }
 
@@ -549,16 +547,16 @@ cudaError_t launch_tc_d(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const
 cudaError_t launch_attention_tc(const void* tm_q, const void* tm_kv, const CacheView& cache,
                                 const BatchView& batch, const WorkItem* items, int n_items,
                                 __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
-                                int g, float scale_log2, int window, int grid, bool exclusive,
+                                int g, float scale_log2, int window, int grid, int sm_end,
                                 int* counter, cudaStream_t stream) {
   if (n_items == 0) return cudaSuccess;
   TcArgs args{cache, batch, items, out, part_o, part_ml, n_q_heads, g, scale_log2, window, n_items,
-              counter};
+              counter, sm_end};
   grid = grid < 1 ? 1 : (grid > n_items ? n_items : grid);
   const CUtensorMap& q = *static_cast<const CUtensorMap*>(tm_q);
   const CUtensorMap& kv = *static_cast<const CUtensorMap*>(tm_kv);
-  if (cache.head_dim == 128) return launch_tc_d<128>(q, kv, args, grid, exclusive, stream);
-  return launch_tc_d<64>(q, kv, args, grid, exclusive, stream);
+  if (cache.head_dim == 128) return launch_tc_d<128>(q, kv, args, grid, stream);
+  return launch_tc_d<64>(q, kv, args, grid, stream);
 }
 
 }  // namespace fg

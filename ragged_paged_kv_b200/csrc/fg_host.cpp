@@ -7,6 +7,7 @@
 // on the host (integer work only) and sends them the same way.
 #include <algorithm>
 #include <chrono>
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -136,7 +137,10 @@ struct fg_ragged_batch {
   int32_t* dmeta = nullptr;
   size_t dmeta_words = 0;
   int32_t* derr = nullptr;
-  int32_t* dctr = nullptr;  // next-unit counters of the persistent kernels
+  // The persistent kernels' next-unit counters sit in the 256 bytes after
+  // the plan in the plan buffer; an upload of a new plan zeroes them too
+  // (ctr_fresh), otherwise a memset does before the kernels run.
+  bool ctr_fresh = false;
   Staging meta_stage;
   // last put
   const fg_kv_cache* cache = nullptr;
@@ -342,7 +346,6 @@ extern "C" fg_status fg_ragged_batch_destroy(fg_ragged_batch* b) {
   b->plan_stage.release();
   if (b->dmeta) cudaFree(b->dmeta);
   if (b->derr) cudaFree(b->derr);
-  if (b->dctr) cudaFree(b->dctr);
   if (b->dplan) cudaFree(b->dplan);
   if (b->ws) cudaFree(b->ws);
   for (cudaEvent_t e : b->tev)
@@ -469,7 +472,6 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
     FG_CUDA(cudaGetDevice(&b->device));
     FG_CUDA(cudaMalloc(&b->dmeta, b->dmeta_words * 4));
     FG_CUDA(cudaMalloc(&b->derr, 4));
-    FG_CUDA(cudaMalloc(&b->dctr, 64));
     FG_CUDA(cudaMemset(b->derr, 0, 4));
     st = b->meta_stage.reserve(b->dmeta_words * 4);
     if (st) return st;
@@ -632,13 +634,37 @@ int sm_count() {
   return n[dev];
 }
 
-// Persistent grids: two CTAs per SM for a kernel that runs alone; one each
-// when the query-tile kernel and a decode kernel share the SMs (a decode CTA
-// then fits beside each query-tile CTA).
-bool overlapped(const fg::Plan& P, bool overlap) {
-  return overlap && P.n_tc > 0 && (P.n_decode > 0 || P.n_dtc > 0);
+// Side-by-side mode: the query-tile kernel (compute bound) takes the SMs with
+// id < K and the tensor-core decode kernel (HBM bound) the rest; decode CTAs
+// also move onto the first K SMs once every query tile has been claimed.
+// K comes from a small cost model: a 128-row x 64-key tile takes about
+// kTileSmUs SM-microseconds (two CTAs per SM), and decode streams about
+// kDecodeSmBytesPerUs per SM up to kHbmBytesPerUs in total (measured on B200).
+// Returns 0 when running the two kernels one after the other is predicted to
+// be as fast.
+constexpr double kTileSmUs = 0.75;
+constexpr double kDecodeSmBytesPerUs = 52.0e3;
+constexpr double kHbmBytesPerUs = 6.4e6;
+
+int tc_share(const fg::Plan& P, int head_dim, int n_sm) {
+  if (P.n_tc == 0 || P.n_dtc == 0 || n_sm < 8) return 0;
+  double tiles = 0.0, bytes = 0.0;
+  for (const WorkItem& w : P.tc) tiles += (w.key_end - (w.key_begin - (w.key_begin & 63)) + 63) / 64;
+  for (const WorkItem& w : P.dtc) bytes += (double)(w.key_end - w.key_begin) * head_dim * 4.0;
+  const double w_tc = tiles * kTileSmUs;
+  auto dec = [&](int sms) { return bytes / std::min(kHbmBytesPerUs, sms * kDecodeSmBytesPerUs); };
+  const double t_seq = w_tc / n_sm + dec(n_sm);
+  int best = 0;
+  double t_best = 0.97 * t_seq;
+  for (int k = 1; k < n_sm; ++k) {
+    const double t = std::max(w_tc / k, dec(n_sm - k));
+    if (t < t_best) {
+      t_best = t;
+      best = k;
+    }
+  }
+  return best;
 }
-int tc_grid(const fg::Plan& P, bool overlap) { return sm_count() * (overlapped(P, overlap) ? 1 : 2); }
 
 fg_status ensure_aux_stream(fg_ragged_batch* b) {
   if (b->aux) return FG_OK;
@@ -665,7 +691,7 @@ fg_status prepare_plan(fg_ragged_batch* b, const fg_kv_cache* c, int32_t g, int3
   fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc,
                  2 * sm_count(), &b->plan);
   b->hprof[4] += now_us() - t_p;
-  const size_t bytes = b->plan.bytes();
+  const size_t bytes = b->plan.bytes() + 256;  // plan, then the unit counters
   if (bytes > b->dplan_bytes) {
     if (b->dplan) FG_CUDA(cudaFreeAsync(b->dplan, strm));
     b->dplan = nullptr;
@@ -682,8 +708,10 @@ fg_status prepare_plan(fg_ragged_batch* b, const fg_kv_cache* c, int32_t g, int3
   b->hprof[5] += now_us() - t_w;
   if (st) return st;
   b->plan.pack(hp);
+  std::memset(static_cast<char*>(hp) + b->plan.bytes(), 0, 256);
   st = b->plan_stage.copy(slot, b->dplan, bytes, strm);
   if (st) return st;
+  b->ctr_fresh = true;
   std::copy(key, key + 4, b->plan_key);
   return FG_OK;
 }
@@ -778,7 +806,8 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   // tensor-core tiles and MHA decode units touch disjoint outputs and
   // partial rows: run them side by side (tc on a high-priority second
   // stream forked from and joined back into the caller's stream)
-  const bool both = overlapped(P, b->overlap);
+  const int tc_sms = b->overlap ? tc_share(P, c->head_dim, sm_count()) : 0;
+  const bool both = tc_sms > 0;
   cudaStream_t tc_stream = strm;
   if (both) {
     st = ensure_aux_stream(b);
@@ -786,7 +815,14 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
     tc_stream = b->aux;
   }
   // the persistent kernels' unit counters start at zero
-  if (P.n_tc || P.n_dtc) FG_CUDA(cudaMemsetAsync(b->dctr, 0, 8, strm));
+  int* ctr = reinterpret_cast<int*>(static_cast<char*>(b->dplan) + P.bytes());
+  if ((P.n_tc || P.n_dtc) && !b->ctr_fresh) FG_CUDA(cudaMemsetAsync(ctr, 0, 8, strm));
+  b->ctr_fresh = false;
+  // programmatic dependent launch along the chain query tiles -> decode ->
+  // combine when the kernels follow each other on one stream with nothing
+  // in between (the decode kernel waits for the query-tile grid before its
+  // CTAs end, so the combine behind it sees both)
+  const bool pdl = !both && !b->timing;
   if (both) {
     FG_CUDA(cudaEventRecord(b->fork, strm));
     FG_CUDA(cudaStreamWaitEvent(b->aux, b->fork, 0));
@@ -795,8 +831,8 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
     if ((st = mark(1, 0, tc_stream))) return st;
     e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
-                                part_ml, n_q_heads, g, scale_log2, window, tc_grid(P, b->overlap),
-                                both, b->dctr, tc_stream);
+                                part_ml, n_q_heads, g, scale_log2, window, 2 * sm_count(),
+                                both ? tc_sms : INT32_MAX, ctr, tc_stream);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
     if ((st = mark(1, 1, tc_stream))) return st;
   }
@@ -811,7 +847,8 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
     e = fg::launch_attention_decode_tc(&tm_q1, &c->tm_kv, cv, b->view,
                                        reinterpret_cast<const WorkItem*>(base + P.off_dtc), P.n_dtc, o,
                                        part_o, part_ml, n_q_heads, g, scale_log2,
-                                       sm_count() * (both ? 1 : 2), b->dctr + 1, strm);
+                                       sm_count() * (both ? 4 : 2), ctr + 1, both ? tc_sms : 0,
+                                       ctr, P.n_tc, pdl && P.n_tc > 0, strm);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core decode launch");
     if ((st = mark(0, 1, strm))) return st;
   }
@@ -822,7 +859,7 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   if (P.n_combine && (st = mark(3, 0, strm))) return st;
   e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),
                          P.n_combine, P.max_combine_rows, part_o, part_ml, o, n_q_heads, g,
-                         c->head_dim, strm);
+                         c->head_dim, pdl && P.n_dtc > 0, strm);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   if (P.n_combine && (st = mark(3, 1, strm))) return st;
   const double t_end = now_us();
@@ -971,7 +1008,7 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
   if (P.n_tc) {
     e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
-                                part_ml, n_q_heads, g, scale_log2, window, 2 * sm_count(), false,
+                                part_ml, n_q_heads, g, scale_log2, window, 2 * sm_count(), INT32_MAX,
                                 ctr, strm);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
   }
@@ -979,12 +1016,12 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
     e = fg::launch_attention_decode_tc(&tm_q1, &c->tm_kv, cv, b->view,
                                        reinterpret_cast<const WorkItem*>(base + P.off_dtc), P.n_dtc, o,
                                        part_o, part_ml, n_q_heads, g, scale_log2, 2 * sm_count(), ctr + 1,
-                                       strm);
+                                       0, nullptr, 0, P.n_tc > 0, strm);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core decode launch");
   }
   e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),
                          P.n_combine, P.max_combine_rows, part_o, part_ml, o, n_q_heads, g,
-                         c->head_dim, strm);
+                         c->head_dim, P.n_dtc > 0, strm);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   return FG_OK;
 }

@@ -88,7 +88,7 @@ cudaError_t launch_attention_decode(const CacheView& cache, const BatchView& bat
 cudaError_t launch_attention_tc(const void* tm_q, const void* tm_kv, const CacheView& cache,
                                 const BatchView& batch, const WorkItem* items, int n_items,
                                 __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
-                                int g, float scale_log2, int window, int grid, bool exclusive,
+                                int g, float scale_log2, int window, int grid, int sm_end,
                                 int* counter, cudaStream_t stream);
 
 // Grouped (or MHA) one-token decode on tensor cores, keys as MMA rows;
@@ -97,11 +97,12 @@ cudaError_t launch_attention_decode_tc(const void* tm_q1, const void* tm_kv, con
                                        const BatchView& batch, const WorkItem* items, int n_items,
                                        __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
                                        int g, float scale_log2, int grid, int* counter,
+                                       int sm_tc_end, const int* tc_counter, int n_tc, bool pdl,
                                        cudaStream_t stream);
 
 cudaError_t launch_combine(const BatchView& batch, const CombineItem* items, int n_items,
                            int max_rows, const float* part_o, const float* part_ml,
-                           __nv_bfloat16* out, int n_q_heads, int g, int head_dim,
+                           __nv_bfloat16* out, int n_q_heads, int g, int head_dim, bool pdl,
                            cudaStream_t stream);
 
 }  // namespace fg
