@@ -11,7 +11,8 @@
 //
 //   warp 4 (TMA)      Q once (3-D box: 64 dims x g heads x 128/g tokens), then
 //                     K and V tiles through the block table, one 2-D box per
-//                     (block part, 64 dims), into 2-stage K and V rings;
+//                     (block part, 64 dims), into 3-stage K and 2-stage V
+//                     rings;
 //   warp 5 (MMA)      one thread issues S = Q K^T into one of two TMEM S
 //                     tiles, and O += P V into the TMEM O tile with P read
 //                     from tensor memory;
@@ -45,7 +46,10 @@ template <int D>
 struct TcCfg {
   static constexpr int BM = 128;  // query rows per tile
   static constexpr int BN = 64;   // keys per tile (two CTAs fit on one SM)
-  static constexpr int KST = 2, VST = 2;
+  // K is needed one tile earlier than V (the S product of tile i is issued
+  // right behind the P.V of tile i-2), so its ring is one stage deeper: at
+  // about 2 us of load latency two stages leave the MMA waiting for K
+  static constexpr int KST = 3, VST = 2;
   static constexpr int DH = D / 64;  // 64-dim (128-byte) boxes per row
   static constexpr int kQBytes = BM * D * 2;
   static constexpr int kKVBytes = BN * D * 2;
@@ -62,6 +66,8 @@ struct TcCfg {
   static constexpr uint32_t kColS = 0;       // S (then P) buffers at columns 0 and BN
   static constexpr uint32_t kColO = 2 * BN;  // O at columns 2*BN .. 2*BN + D
   static_assert(kColO + D <= kTmemCols, "TMEM budget");
+  // two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA
+  static_assert(2 * (kSmem + 1024) <= 228 * 1024, "two CTAs must fit on one SM");
 };
 
 struct TcArgs {
@@ -167,9 +173,9 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
   uint64_t* uq_full = o_free + 1;
   uint64_t* uq_empty = uq_full + UnitQueue::kDepth;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
-  // units come from a global counter through this queue (MMA thread and the
-  // four softmax warps consume)
-  const UnitQueue uq{reinterpret_cast<int32_t*>(tmem_slot + 4), uq_full, uq_empty, 5};
+  // units come from a global counter through this queue (the V loader, the
+  // MMA thread and the four softmax warps consume)
+  const UnitQueue uq{reinterpret_cast<int32_t*>(tmem_slot + 4), uq_full, uq_empty, 6};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = a.g;
@@ -207,24 +213,39 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
 
   if (warp == 4) {
     // ---------------------------------------------------------------- TMA
-    if (lane == 0) {
+    // Lane 0 takes units from the global counter and loads Q and the K
+    // tiles; lane 1 follows the same units through the queue and loads the
+    // V tiles. The two streams run on independent rings, so a K load is
+    // never held back behind a V stage that the P.V of an earlier tile still
+    // occupies.
+    if (lane < 2) {
+      const bool is_k = lane == 0;
       const int B = a.cache.block_size;
       const int BR = B < 64 ? B : 64;
       const int Hkv = a.cache.n_kv_heads;
+      const int kv = is_k ? 0 : 1;
+      const int NST = is_k ? C::KST : C::VST;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      unsigned char* ring = is_k ? sK : sV;
       int gt = 0, un = 0;
       for (;; ++un) {
         int u = -1;
-        if (!uq.push_next(un, a.counter, a.n_items, kWaitLimit, &u)) {
+        const bool got = is_k ? uq.push_next(un, a.counter, a.n_items, kWaitLimit, &u)
+                              : uq.pop(un, false, kWaitLimit, &u);
+        if (!got) {
           atomicOr(err, kErrTimeout);
           ok = false;
         }
         if (u < 0 || !ok) break;
         const Unit x = load_unit(a, u, C::BN);
-        if (un >= 1 && !wait_or_flag(q_empty, (un - 1) & 1, err, ok)) break;
-        ptx::mbar_arrive_expect_tx(q_full, C::kQBytes);
+        if (is_k) {
+          if (un >= 1 && !wait_or_flag(q_empty, (un - 1) & 1, err, ok)) break;
+          ptx::mbar_arrive_expect_tx(q_full, C::kQBytes);
 #pragma unroll
-        for (int dh = 0; dh < C::DH; ++dh)
-          ptx::tma_load_3d(sQ + dh * C::BM * 128, &tm_q, dh * 64, x.h * g, x.row0, q_full);
+          for (int dh = 0; dh < C::DH; ++dh)
+            ptx::tma_load_3d(sQ + dh * C::BM * 128, &tm_q, dh * 64, x.h * g, x.row0, q_full);
+        }
         const int32_t* bt = a.batch.bt + a.batch.bt_off[x.s];
         const int nb = a.batch.bt_off[x.s + 1] - a.batch.bt_off[x.s];
         for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
@@ -234,47 +255,31 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
             const int lb = pos / B;
             if (lb < nb && bt[lb] >= 0 && bt[lb] < a.cache.n_blocks) bytes += BR * 128 * C::DH;
           }
-          const int ks = gt % C::KST, vs = gt % C::VST;
-          if (gt >= C::KST && !wait_or_flag(&k_empty[ks], ((gt / C::KST) - 1) & 1, err, ok)) break;
-          ptx::mbar_arrive_expect_tx(&k_full[ks], bytes);
+          const int st = gt % NST;
+          if (gt >= NST && !wait_or_flag(&empty[st], ((gt / NST) - 1) & 1, err, ok)) break;
+          ptx::mbar_arrive_expect_tx(&full[st], bytes);
           for (int pos = k0; pos < k0 + C::BN; pos += BR) {
             const int lb = pos / B;
             if (lb >= nb) continue;
             const int32_t blk = bt[lb];
             if (blk < 0 || blk >= a.cache.n_blocks) {
-              atomicOr(err, kErrBadBlock);
+              if (is_k) atomicOr(err, kErrBadBlock);
               continue;
             }
-            const int row = (int)(((int64_t)blk * 2 * Hkv + x.h) * B + (pos - lb * B));
+            const int row = (int)((((int64_t)blk * 2 + kv) * Hkv + x.h) * B + (pos - lb * B));
 #pragma unroll
             for (int dh = 0; dh < C::DH; ++dh)
-              ptx::tma_load_2d(sK + ks * C::kKVBytes + dh * C::BN * 128 + (pos - k0) * 128, &tm_kv,
-                               dh * 64, row, &k_full[ks]);
-          }
-          if (gt >= C::VST && !wait_or_flag(&v_empty[vs], ((gt / C::VST) - 1) & 1, err, ok)) break;
-          ptx::mbar_arrive_expect_tx(&v_full[vs], bytes);
-          for (int pos = k0; pos < k0 + C::BN; pos += BR) {
-            const int lb = pos / B;
-            if (lb >= nb) continue;
-            const int32_t blk = bt[lb];
-            if (blk < 0 || blk >= a.cache.n_blocks) continue;
-            const int row = (int)((((int64_t)blk * 2 + 1) * Hkv + x.h) * B + (pos - lb * B));
-#pragma unroll
-            for (int dh = 0; dh < C::DH; ++dh)
-              ptx::tma_load_2d(sV + vs * C::kKVBytes + dh * C::BN * 128 + (pos - k0) * 128, &tm_kv,
-                               dh * 64, row, &v_full[vs]);
+              ptx::tma_load_2d(ring + st * C::kKVBytes + dh * C::BN * 128 + (pos - k0) * 128, &tm_kv, dh * 64,
+                               row, &full[st]);
           }
         }
       }
       // every unit is claimed: a grid launched behind this one (the decode
       // kernel) may take SMs as this kernel's CTAs leave
-      ptx::allow_dependent_launch();
+      if (is_k) ptx::allow_dependent_launch();
       // let in-flight loads land before the CTA can exit
-      for (int t = max(0, gt - C::KST); t < gt && ok; ++t)
-        wait_or_flag(&k_full[t % C::KST], (t / C::KST) & 1, err, ok);
-      for (int t = max(0, gt - C::VST); t < gt && ok; ++t)
-        wait_or_flag(&v_full[t % C::VST], (t / C::VST) & 1, err, ok);
-      if (un >= 1) wait_or_flag(q_full, (un - 1) & 1, err, ok);
+      for (int t = max(0, gt - NST); t < gt && ok; ++t) wait_or_flag(&full[t % NST], (t / NST) & 1, err, ok);
+      if (is_k && un >= 1) wait_or_flag(q_full, (un - 1) & 1, err, ok);
     }
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA
