@@ -1,29 +1,38 @@
 // Ragged paged attention on the 5th-generation tensor cores (tcgen05).
 //
-// A work unit is one 128-row query tile of one sequence and kv head: the
-// rows are (token, q head of the group) pairs, 128/g consecutive new tokens
-// times the g q heads that share the kv head, so a grouped-query tile reuses
-// each K/V tile for all g heads. The kernel is persistent: the TMA warp takes
-// units one by one from a global counter over a longest-first list and hands
-// them to the other warps, and every role counts tiles globally, so the rings
-// and barrier phases run on across units (the next unit's K/V stream in while
-// the last one's epilogue runs). A unit walks its key range in 64-key tiles:
+// A work unit is up to two 128-row query tiles (0 and 1) of one sequence and
+// kv head that share every K/V tile: the rows are (token, q head of the
+// group) pairs, up to 256/g consecutive new tokens times the g q heads that
+// share the kv head, rows 0-127 in tile 0 and 128-255 in tile 1. Each K/V
+// tile is loaded once per unit and serves both query tiles and all g heads.
+// The kernel is persistent, one CTA per SM: the K loader takes units one by
+// one from a global counter over a longest-first list and hands them to the
+// other roles, and every role counts tiles globally, so the rings and barrier
+// phases run on across units. A unit walks the key range of its last row in
+// 64-key tiles:
 //
-//   warp 4 (TMA)      Q once (3-D box: 64 dims x g heads x 128/g tokens), then
-//                     K and V tiles through the block table, one 2-D box per
-//                     (block part, 64 dims), into 3-stage K and 2-stage V
-//                     rings;
-//   warp 5 (MMA)      one thread issues S = Q K^T into one of two TMEM S
-//                     tiles, and O += P V into the TMEM O tile with P read
-//                     from tensor memory;
-//   warps 0-3         thread r owns query row r (TMEM lane r): reads its S
-//                     row with tcgen05.ld, masks (causal, window, unit range),
+//   warp 8, lane 0    Q of both query tiles once per unit (3-D boxes: 64
+//                     dims x g heads x 128/g tokens), then K tiles through the
+//                     block table into a 5-stage ring;
+//   warp 8, lane 1    V tiles, the same way, into a 4-stage ring (separate
+//                     streams, so a K load never waits behind a V stage that
+//                     an earlier P.V still occupies);
+//   warps 9, 10 (MMA) one thread per query tile issues S_t = Q_t K^T into
+//                     double-buffered TMEM S tiles and O_t += P_t V into its
+//                     TMEM O tile, with P read from tensor memory; the two
+//                     tiles' pipelines only meet at the shared K/V rings;
+//   warps 0-3 / 4-7   softmax of query tile 0 / 1: thread r of a warpgroup
+//                     owns row r of its tile (TMEM lane r): reads its S row
+//                     with tcgen05.ld, masks (causal, window, unit range),
 //                     keeps an online softmax (a running max that is only
 //                     moved - with a rescale of its O row in TMEM - when a
 //                     tile raises it by more than 2^8), writes P as packed
 //                     bf16 back over the S tile it came from, and at the end
 //                     normalises O and stores it.
 //
+// Sharing K/V between two query tiles halves the K/V traffic from L2 per
+// flop and leaves shared memory for deep rings; the two softmax warpgroups
+// keep the tensor core fed while each works through its exponentials.
 // Keeping P in tensor memory makes it double-buffered with S for free: the
 // softmax of tile i+1 never waits for the P.V product of tile i, and the S
 // product of tile i+2, which overwrites that buffer, is issued right behind
@@ -45,29 +54,27 @@ constexpr long long kWaitLimit = 1LL << 31;
 template <int D>
 struct TcCfg {
   static constexpr int BM = 128;  // query rows per tile
-  static constexpr int BN = 64;   // keys per tile (two CTAs fit on one SM)
-  // K is needed one tile earlier than V (the S product of tile i is issued
-  // right behind the P.V of tile i-2), so its ring is one stage deeper: at
-  // about 2 us of load latency two stages leave the MMA waiting for K
-  static constexpr int KST = 3, VST = 2;
+  static constexpr int NQ = 2;    // query tiles per unit
+  static constexpr int BN = 64;   // keys per K/V tile
+  static constexpr int KST = 5, VST = 4;
   static constexpr int DH = D / 64;  // 64-dim (128-byte) boxes per row
   static constexpr int kQBytes = BM * D * 2;
   static constexpr int kKVBytes = BN * D * 2;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffK = kOffQ + NQ * kQBytes;
   static constexpr int kOffV = kOffK + KST * kKVBytes;
   static constexpr int kOffBar = kOffV + VST * kKVBytes;
   // q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST],
-  // s_full[2], p_full[2], pv_done[2], o_free, unit queue full/empty
-  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 2 * UnitQueue::kDepth;
+  // then per query tile: s_full[2], p_full[2], pv_done[2], o_free; unit queue
+  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + NQ * 7 + 2 * UnitQueue::kDepth;
   static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + UnitQueue::kDepth * 4;
-  static constexpr int kThreads = 192;
-  static constexpr uint32_t kTmemCols = 256;
-  static constexpr uint32_t kColS = 0;       // S (then P) buffers at columns 0 and BN
-  static constexpr uint32_t kColO = 2 * BN;  // O at columns 2*BN .. 2*BN + D
-  static_assert(kColO + D <= kTmemCols, "TMEM budget");
-  // two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA
-  static_assert(2 * (kSmem + 1024) <= 228 * 1024, "two CTAs must fit on one SM");
+  static constexpr int kThreads = 352;  // 8 softmax warps, the load warp, one MMA warp per query tile
+  static constexpr uint32_t kTmemCols = 512;
+  // query tile t: S (then P) buffers at kColS0 + 2 t BN and + BN, O at kColO0 + t D
+  static constexpr uint32_t kColS0 = 0;
+  static constexpr uint32_t kColO0 = NQ * 2 * BN;
+  static_assert(kColO0 + NQ * D <= kTmemCols, "TMEM budget");
+  static_assert(kSmem + 1024 <= 228 * 1024, "shared memory budget");
 };
 
 struct TcArgs {
@@ -143,7 +150,7 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+__global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                         const __grid_constant__ CUtensorMap tm_kv,
                                                         TcArgs a) {
   using C = TcCfg<D>;
@@ -166,16 +173,17 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
   uint64_t* k_empty = k_full + C::KST;
   uint64_t* v_full = k_empty + C::KST;
   uint64_t* v_empty = v_full + C::VST;
-  uint64_t* s_full = v_empty + C::VST;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
-  uint64_t* o_free = pv_done + 2;
-  uint64_t* uq_full = o_free + 1;
+  uint64_t* tb = v_empty + C::VST;  // query tile t: 7 barriers from tb + 7 t
+  auto s_full = [tb](int t, int b) { return tb + 7 * t + b; };
+  auto p_full = [tb](int t, int b) { return tb + 7 * t + 2 + b; };
+  auto pv_done = [tb](int t, int b) { return tb + 7 * t + 4 + b; };
+  auto o_free = [tb](int t) { return tb + 7 * t + 6; };
+  uint64_t* uq_full = tb + 7 * C::NQ;
   uint64_t* uq_empty = uq_full + UnitQueue::kDepth;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   // units come from a global counter through this queue (the V loader, the
-  // MMA thread and the four softmax warps consume)
-  const UnitQueue uq{reinterpret_cast<int32_t*>(tmem_slot + 4), uq_full, uq_empty, 6};
+  // two MMA threads and the eight softmax warps consume)
+  const UnitQueue uq{reinterpret_cast<int32_t*>(tmem_slot + 4), uq_full, uq_empty, 11};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = a.g;
@@ -183,25 +191,28 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(q_full, 1);
-    ptx::mbar_init(q_empty, 1);
+    // Q and every K/V stage are released by both MMA threads
+    ptx::mbar_init(q_empty, C::NQ);
     for (int i = 0; i < C::KST; ++i) {
       ptx::mbar_init(&k_full[i], 1);
-      ptx::mbar_init(&k_empty[i], 1);
+      ptx::mbar_init(&k_empty[i], C::NQ);
     }
     for (int i = 0; i < C::VST; ++i) {
       ptx::mbar_init(&v_full[i], 1);
-      ptx::mbar_init(&v_empty[i], 1);
+      ptx::mbar_init(&v_empty[i], C::NQ);
     }
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&s_full[i], 1);
-      ptx::mbar_init(&p_full[i], 4);
-      ptx::mbar_init(&pv_done[i], 1);
+    for (int t = 0; t < C::NQ; ++t) {
+      for (int i = 0; i < 2; ++i) {
+        ptx::mbar_init(s_full(t, i), 1);
+        ptx::mbar_init(p_full(t, i), 4);
+        ptx::mbar_init(pv_done(t, i), 1);
+      }
+      ptx::mbar_init(o_free(t), 4);
     }
-    ptx::mbar_init(o_free, 4);
     uq.init();
     ptx::fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tmem_alloc(tmem_slot, C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -211,13 +222,8 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
-  if (warp == 4) {
-    // ---------------------------------------------------------------- TMA
-    // Lane 0 takes units from the global counter and loads Q and the K
-    // tiles; lane 1 follows the same units through the queue and loads the
-    // V tiles. The two streams run on independent rings, so a K load is
-    // never held back behind a V stage that the P.V of an earlier tile still
-    // occupies.
+  if (warp == 8) {
+    // ---------------------------------------------------------------- loads
     if (lane < 2) {
       const bool is_k = lane == 0;
       const int B = a.cache.block_size;
@@ -240,11 +246,16 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
         if (u < 0 || !ok) break;
         const Unit x = load_unit(a, u, C::BN);
         if (is_k) {
+          // both query tiles' boxes (tile 1's reaches past the unit's rows
+          // when R <= 128; those rows are never used)
           if (un >= 1 && !wait_or_flag(q_empty, (un - 1) & 1, err, ok)) break;
-          ptx::mbar_arrive_expect_tx(q_full, C::kQBytes);
+          ptx::mbar_arrive_expect_tx(q_full, C::NQ * C::kQBytes);
 #pragma unroll
-          for (int dh = 0; dh < C::DH; ++dh)
-            ptx::tma_load_3d(sQ + dh * C::BM * 128, &tm_q, dh * 64, x.h * g, x.row0, q_full);
+          for (int t = 0; t < C::NQ; ++t)
+#pragma unroll
+            for (int dh = 0; dh < C::DH; ++dh)
+              ptx::tma_load_3d(sQ + t * C::kQBytes + dh * C::BM * 128, &tm_q, dh * 64, x.h * g,
+                               x.row0 + t * (C::BM / g), q_full);
         }
         const int32_t* bt = a.batch.bt + a.batch.bt_off[x.s];
         const int nb = a.batch.bt_off[x.s + 1] - a.batch.bt_off[x.s];
@@ -281,32 +292,35 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
       for (int t = max(0, gt - NST); t < gt && ok; ++t) wait_or_flag(&full[t % NST], (t / NST) & 1, err, ok);
       if (is_k && un >= 1) wait_or_flag(q_full, (un - 1) & 1, err, ok);
     }
-  } else if (warp == 5) {
+  } else if (warp >= 9) {
     // ---------------------------------------------------------------- MMA
+    // One thread per query tile, so the two tiles' pipelines only meet at
+    // the shared K/V rings: each thread walks every unit and K/V tile,
+    // issues its tile's S and P.V products, and releases Q and each K/V
+    // stage once (with a plain arrival when its tile has no rows).
     if (lane == 0) {
+      const int t = warp - 9;
       constexpr uint32_t idesc_qk = ptx::idesc_bf16_f32(C::BM, C::BN, 0, 0);
       constexpr uint32_t idesc_pv = ptx::idesc_bf16_f32(C::BM, D, 0, 1);
-      const uint32_t q_addr = ptx::smem_u32(sQ), k_addr = ptx::smem_u32(sK);
+      const uint32_t q_addr = ptx::smem_u32(sQ) + t * C::kQBytes, k_addr = ptx::smem_u32(sK);
       const uint32_t v_addr = ptx::smem_u32(sV);
-      int gt = 0, un = 0;
-      // O += P V for global tile t, P in the TMEM S buffer t&1 (bf16 packed,
-      // 16 keys = 8 columns per MMA step); `first` starts a unit's
-      // accumulation and must wait until the previous unit's epilogue has
-      // read O.
-      auto issue_pv = [&](int t, bool first) {
-        const int vs = t % C::VST, pb = t & 1;
-        if (!wait_or_flag(&v_full[vs], (t / C::VST) & 1, err, ok)) return;
-        if (!wait_or_flag(&p_full[pb], (t >> 1) & 1, err, ok)) return;
-        if (first && un >= 1 && !wait_or_flag(o_free, (un - 1) & 1, err, ok)) return;
+      const uint32_t col_s = C::kColS0 + t * 2 * C::BN, col_o = C::kColO0 + t * D;
+      int gt = 0, un = 0, ns = 0, np = 0, nu = 0;
+      // O_t += P_t V for the tile's next P (TMEM S buffer np & 1, bf16
+      // packed, 16 keys = 8 columns per MMA step); `first` starts a unit's
+      // accumulation and must wait until this tile's previous epilogue has
+      // read O_t.
+      auto issue_pv = [&](int vs, bool first) {
+        const int l = np++, pb = l & 1;
+        if (!wait_or_flag(p_full(t, pb), (l >> 1) & 1, err, ok)) return;
+        if (first && nu >= 2 && !wait_or_flag(o_free(t), (nu - 2) & 1, err, ok)) return;
         ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           const uint64_t bd = ptx::smem_desc_sw128(v_addr + vs * C::kKVBytes + kk * 16 * 128, C::BN * 128, 1024);
-          mma_bf16_ts(tmem + C::kColO, tmem + C::kColS + pb * C::BN + kk * 8, bd, idesc_pv,
-                      (!first || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + col_o, tmem + col_s + pb * C::BN + kk * 8, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
         }
-        ptx::mma_commit(&pv_done[pb]);
-        ptx::mma_commit(&v_empty[vs]);
+        ptx::mma_commit(pv_done(t, pb));
       };
       for (;; ++un) {
         int u = -1;
@@ -316,37 +330,64 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
         }
         if (u < 0 || !ok) break;
         const Unit x = load_unit(a, u, C::BN);
+        const bool live = x.R > t * C::BM;
+        if (!live) {
+          // nothing to compute: release Q and the unit's K/V stages as they
+          // fill (the loaders' phases must see this thread's arrivals)
+          if (!wait_or_flag(q_full, un & 1, err, ok)) break;
+          ptx::mbar_arrive(q_empty);
+          for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
+            if (!wait_or_flag(&k_full[gt % C::KST], (gt / C::KST) & 1, err, ok)) break;
+            ptx::mbar_arrive(&k_empty[gt % C::KST]);
+            if (!wait_or_flag(&v_full[gt % C::VST], (gt / C::VST) & 1, err, ok)) break;
+            ptx::mbar_arrive(&v_empty[gt % C::VST]);
+          }
+          continue;
+        }
+        ++nu;
         if (!wait_or_flag(q_full, un & 1, err, ok)) break;
-        const int gt0 = gt;
         for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
-          const int ks = gt % C::KST, sb = gt & 1;
+          const int ks = gt % C::KST;
           if (!wait_or_flag(&k_full[ks], (gt / C::KST) & 1, err, ok)) break;
-          // S buffer sb holds P of tile gt-2, which the P.V product issued
-          // just before this one reads: tcgen05.mma operations issued by one
-          // thread execute in issue order, so this S product is queued
-          // behind that P.V instead of waiting for its completion here
           ptx::tc_fence_after();
+          // S buffer sb holds P of this tile's tile ns - 2, which the P.V
+          // issued earlier reads: the tensor core runs this thread's MMAs in
+          // issue order, so this S product queues behind it
+          const int sb = ns++ & 1;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::BM * 128 + (kk & 3) * 32;
             const uint64_t ad = ptx::smem_desc_sw128(q_addr + off, 16, 1024);
             const uint64_t bd = ptx::smem_desc_sw128(
                 k_addr + ks * C::kKVBytes + (kk >> 2) * C::BN * 128 + (kk & 3) * 32, 16, 1024);
-            ptx::mma_bf16(tmem + C::kColS + sb * C::BN, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+            ptx::mma_bf16(tmem + col_s + sb * C::BN, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
           }
-          ptx::mma_commit(&s_full[sb]);
+          ptx::mma_commit(s_full(t, sb));
           ptx::mma_commit(&k_empty[ks]);
           if (i == x.n_tiles - 1) ptx::mma_commit(q_empty);
-          if (i >= 1) issue_pv(gt - 1, i == 1);
+          if (i >= 1) {
+            const int vs = (gt - 1) % C::VST;
+            if (!wait_or_flag(&v_full[vs], ((gt - 1) / C::VST) & 1, err, ok)) break;
+            issue_pv(vs, i == 1);
+            ptx::mma_commit(&v_empty[vs]);
+          }
         }
-        if (ok) issue_pv(gt - 1, gt - 1 == gt0);
+        if (ok) {
+          const int vs = (gt - 1) % C::VST;
+          if (wait_or_flag(&v_full[vs], ((gt - 1) / C::VST) & 1, err, ok)) {
+            issue_pv(vs, x.n_tiles == 1);
+            ptx::mma_commit(&v_empty[vs]);
+          }
+        }
       }
     }
   } else {
     // ---------------------------------------------------- softmax / epilogue
-    const int r = threadIdx.x;  // query row == TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    int gt = 0, un = 0;
+    const int qt = warp >> 2;              // query tile of this warpgroup
+    const int r = (warp & 3) * 32 + lane;  // row within the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t col_s = C::kColS0 + qt * 2 * C::BN, col_o = C::kColO0 + qt * D;
+    int gt = 0, lt = 0, un = 0;  // global K/V tiles; tiles of this query tile; units
     for (;; ++un) {
       int u = -1;
       if (!uq.pop(un, true, kWaitLimit, &u)) {
@@ -355,30 +396,33 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
       }
       if (u < 0 || !ok) break;
       const Unit x = load_unit(a, u, C::BN);
-      const bool row_ok = r < x.R;
-      const int p_r = x.ctx + x.tok_begin + r / g;
+      if (x.R <= qt * C::BM) {  // this query tile has no rows in the unit
+        gt += x.n_tiles;
+        continue;
+      }
+      const int rr = qt * C::BM + r;  // row within the unit
+      const bool row_ok = rr < x.R;
+      const int p_r = x.ctx + x.tok_begin + rr / g;
       int lower = 0, upper = 0;
       if (row_ok) {
         lower = max(x.kb, a.window > 0 ? p_r - a.window + 1 : 0);
         upper = min(x.ke, p_r + 1);
       }
-      const bool warp_live = (warp * 32) < x.R;
+      const bool warp_live = qt * C::BM + (warp & 3) * 32 < x.R;
       float m_used = -INFINITY, l = 0.f;
-      for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
-        const int sb = gt & 1;
+      for (int i = 0; i < x.n_tiles && ok; ++i, ++lt, ++gt) {
+        const int sb = lt & 1;
         const int k0 = x.k00 + i * C::BN;
-        if (!wait_or_flag(&s_full[sb], (gt >> 1) & 1, err, ok)) break;
+        if (!wait_or_flag(s_full(qt, sb), (lt >> 1) & 1, err, ok)) break;
         if (warp_live) {
           ptx::tc_fence_after();
           uint32_t raw[C::BN];
 #pragma unroll
           for (int c = 0; c < C::BN / 32; ++c)
-            ptx::tmem_ld32(tmem + lane_base + C::kColS + sb * C::BN + c * 32,
+            ptx::tmem_ld32(tmem + lane_base + col_s + sb * C::BN + c * 32,
                            *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
           ptx::tmem_ld_wait();
           float sv[C::BN];
-          // mask, then the tile max as a tree of 3-input maxima (8 independent
-          // chains, so the reduction is not one 64-long dependency chain)
           const int c_lo = lower - k0, c_hi = upper - k0;
 #pragma unroll
           for (int c = 0; c < C::BN; ++c) sv[c] = __uint_as_float(raw[c]);
@@ -389,6 +433,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
             for (int c = 0; c < C::BN; ++c)
               if (c < c_lo || c >= c_hi) sv[c] = -INFINITY;
           }
+          // the tile max as a tree of 3-input maxima (8 independent chains)
           float mx[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) mx[j] = fmaxf(sv[j], sv[8 + j]);
@@ -406,31 +451,30 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
           }
           // O may be rescaled only once the P.V of the previous tile is done
           if (i >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-            if (!wait_or_flag(&pv_done[(gt - 1) & 1], ((gt - 1) >> 1) & 1, err, ok)) break;
+            if (!wait_or_flag(pv_done(qt, (lt - 1) & 1), ((lt - 1) >> 1) & 1, err, ok)) break;
             ptx::tc_fence_after();
+            const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
-              const uint32_t ta = tmem + lane_base + C::kColO + c * 32;
+              const uint32_t ta = tmem + lane_base + col_o + c * 32;
               ptx::tmem_ld32(ta, o);
               ptx::tmem_ld_wait();
-              const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
               for (int e = 0; e < 32; e += 2) {
-                const float2 r = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), al2);
-                o[e] = __float_as_uint(r.x);
-                o[e + 1] = __float_as_uint(r.y);
+                const float2 v2 = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), al2);
+                o[e] = __float_as_uint(v2.x);
+                o[e + 1] = __float_as_uint(v2.y);
               }
               ptx::tmem_st32(ta, o);
             }
             ptx::tmem_st_wait();
           }
           // P = 2^(s*scale - m_used), packed two bf16 per 32-bit word, written
-          // over the first BN/2 columns of this S buffer (lane r = row r).
-          // Masked keys are -inf and give 0; a row with no key yet has
-          // m_used = -inf, all its scores -inf, and neg_m = 0 keeps them 0.
+          // over the first BN/2 columns of this S buffer (lane r = row r);
           // the scale-and-shift and the running sums use the packed f32x2
-          // FMA/add, two keys per instruction
+          // FMA/add. Masked keys are -inf and give 0; a row with no key yet
+          // has m_used = -inf, all its scores -inf, and neg_m = 0 keeps them 0.
           float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                           make_float2(0.f, 0.f)};
           const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
@@ -438,26 +482,28 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
           uint32_t pw[C::BN / 2];
 #pragma unroll
           for (int c = 0; c < C::BN / 2; ++c) {
-            const float2 x = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
-            const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+            const float2 xx = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
+            const float2 pp = make_float2(ex2(xx.x), ex2(xx.y));
             ls[c & 3] = __fadd2_rn(ls[c & 3], pp);
             __nv_bfloat162 pr = __floats2bfloat162_rn(pp.x, pp.y);
             pw[c] = *reinterpret_cast<uint32_t*>(&pr);
           }
-          ptx::tmem_st32(tmem + lane_base + C::kColS + sb * C::BN, pw);
+          ptx::tmem_st32(tmem + lane_base + col_s + sb * C::BN, pw);
           const float2 l01 = __fadd2_rn(ls[0], ls[1]), l23 = __fadd2_rn(ls[2], ls[3]);
           l += (l01.x + l01.y) + (l23.x + l23.y);
           // keys at or past the sequence end may hold anything (unwritten
           // slots, stale stage data): zero those V rows so 0 * garbage cannot
-          // reach O
+          // reach O. Both warpgroups may do it for a stage (the same zeros),
+          // each before its own P.V can be issued.
           if (k0 + C::BN > x.L) {
             const int vs = gt % C::VST;
             if (!wait_or_flag(&v_full[vs], (gt / C::VST) & 1, err, ok)) break;
             const int z0 = max(0, x.L - k0);
             const int per_dh = (C::BN - z0) * 8;  // 16-byte chunks per 64-dim half
             const int nz = per_dh * C::DH;
-            const int n_live = min(C::BM, (x.R + 31) & ~31);  // threads of the live warps
-            for (int z = threadIdx.x; z < nz; z += n_live) {
+            const int live_rows = min(C::BM, x.R - qt * C::BM);
+            const int n_live = (live_rows + 31) & ~31;  // threads of the warpgroup's live warps
+            for (int z = r; z < nz; z += n_live) {
               const int dh = z / per_dh, rem = z - dh * per_dh;
               const int row = z0 + rem / 8, chn = rem % 8;
               *reinterpret_cast<uint4*>(sV + vs * C::kKVBytes + dh * C::BN * 128 + row * 128 + chn * 16) =
@@ -468,24 +514,24 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
           ptx::tmem_st_wait();
         }
         // padding warps write no P: arriving right after their s_full wait
-        // is safe, because tile gt + 2 cannot start before this phase ends
+        // is safe, because tile lt + 2 cannot start before this phase ends
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&p_full[sb]);
+        if (lane == 0) ptx::mbar_arrive(p_full(qt, sb));
       }
       if (!ok) break;
       // epilogue: wait for the unit's last PV, normalise, store, free O
-      const int last = gt - 1;
-      if (!wait_or_flag(&pv_done[last & 1], (last >> 1) & 1, err, ok)) break;
+      const int last = lt - 1;
+      if (!wait_or_flag(pv_done(qt, last & 1), (last >> 1) & 1, err, ok)) break;
       ptx::tc_fence_after();
       if (warp_live) {
-        const int row = x.row0 + r / g;
-        const int qh = x.h * g + (r % g);
+        const int row = x.row0 + rr / g;
+        const int qh = x.h * g + (rr % g);
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          ptx::tmem_ld32(tmem + lane_base + C::kColO + c * 32, o);
+          ptx::tmem_ld32(tmem + lane_base + col_o + c * 32, o);
           ptx::tmem_ld_wait();
           if (!row_ok) continue;
           if (x.part < 0) {
@@ -502,7 +548,7 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
               dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(a.part_o + (int64_t)(x.part + r) * D + c * 32);
+            float4* dst = reinterpret_cast<float4*>(a.part_o + (int64_t)(x.part + rr) * D + c * 32);
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4)
               dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
@@ -510,18 +556,18 @@ __global__ void __launch_bounds__(192, 2) attn_tc_kernel(const __grid_constant__
           }
         }
         if (row_ok && x.part >= 0) {
-          a.part_ml[(int64_t)(x.part + r) * 2] = m_used;
-          a.part_ml[(int64_t)(x.part + r) * 2 + 1] = l;
+          a.part_ml[(int64_t)(x.part + rr) * 2] = m_used;
+          a.part_ml[(int64_t)(x.part + rr) * 2 + 1] = l;
         }
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(o_free);
+      if (lane == 0) ptx::mbar_arrive(o_free(qt));
     }
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -536,8 +582,6 @@ cudaError_t launch_tc_d(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const
     cudaError_t e =
         cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
-    // the largest shared-memory carveout: two CTAs per SM, and a decode CTA
-    // beside one when the kernels share the GPU
     e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;

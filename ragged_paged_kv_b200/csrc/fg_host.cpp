@@ -649,7 +649,8 @@ constexpr double kHbmBytesPerUs = 6.4e6;
 int tc_share(const fg::Plan& P, int head_dim, int n_sm) {
   if (P.n_tc == 0 || P.n_dtc == 0 || n_sm < 8) return 0;
   double tiles = 0.0, bytes = 0.0;
-  for (const WorkItem& w : P.tc) tiles += (w.key_end - (w.key_begin - (w.key_begin & 63)) + 63) / 64;
+  for (const WorkItem& w : P.tc)
+    tiles += ((w.key_end - (w.key_begin - (w.key_begin & 63)) + 63) / 64) * (w.n_rows > fg::kTcRows ? 2 : 1);
   for (const WorkItem& w : P.dtc) bytes += (double)(w.key_end - w.key_begin) * head_dim * 4.0;
   const double w_tc = tiles * kTileSmUs;
   auto dec = [&](int sms) { return bytes / std::min(kHbmBytesPerUs, sms * kDecodeSmBytesPerUs); };
@@ -689,7 +690,7 @@ fg_status prepare_plan(fg_ragged_batch* b, const fg_kv_cache* c, int32_t g, int3
   if (std::equal(key, key + 4, b->plan_key) && b->dplan) return FG_OK;
   const double t_p = now_us();
   fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc,
-                 2 * sm_count(), &b->plan);
+                 sm_count(), &b->plan);
   b->hprof[4] += now_us() - t_p;
   const size_t bytes = b->plan.bytes() + 256;  // plan, then the unit counters
   if (bytes > b->dplan_bytes) {
@@ -831,7 +832,7 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
     if ((st = mark(1, 0, tc_stream))) return st;
     e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
-                                part_ml, n_q_heads, g, scale_log2, window, 2 * sm_count(),
+                                part_ml, n_q_heads, g, scale_log2, window, sm_count(),
                                 both ? tc_sms : INT32_MAX, ctr, tc_stream);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
     if ((st = mark(1, 1, tc_stream))) return st;
@@ -976,7 +977,7 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
   thread_local fg::Plan P;
   thread_local std::vector<unsigned char> packed;
   fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc,
-                 2 * sm_count(), &P);
+                 sm_count(), &P);
   // the last 256 bytes of the plan area hold the persistent kernels' counters
   if (P.bytes() + 256 > plan_bytes)
     return fail(FG_ERR_CAPACITY, "pass needs a %zu-byte work plan, the fixed area holds %zu",
@@ -1008,7 +1009,7 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
   if (P.n_tc) {
     e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
-                                part_ml, n_q_heads, g, scale_log2, window, 2 * sm_count(), INT32_MAX,
+                                part_ml, n_q_heads, g, scale_log2, window, sm_count(), INT32_MAX,
                                 ctr, strm);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
   }

@@ -71,7 +71,7 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
       continue;
     }
     if (use_tc) {
-      const int tpt = kTcRows / g;
+      const int tpt = kTcUnitRows / g;
       // Few long query tiles leave persistent CTAs idle at the end: then
       // tiles of >= 2 * kTcMinSplitKeys keys are cut into pieces of at least
       // kTcMinSplitKeys keys so that there are about 4 units per CTA slot.

@@ -14,6 +14,7 @@ constexpr int kGeneralRows = 16;  // query rows per general-path unit
 constexpr int kSplitKeys = 1024;  // keys per split-KV partial (general path)
 constexpr int kDecodeSplitKeys = 512;  // keys per unit of the MHA decode kernel
 constexpr int kTcRows = 128;           // query rows per tensor-core tile
+constexpr int kTcUnitRows = 256;       // query rows per tensor-core unit (two tiles sharing K/V)
 constexpr int kTcDecodeSplitKeys = 2048;  // keys per unit for small (decode) tc tiles
 constexpr int kDtcMaxGroup = 16;          // q heads per kv head the decode tc kernel serves
 constexpr int kTcMinSplitKeys = 4096;     // shortest piece when a long query tile is split
@@ -47,7 +48,7 @@ struct Plan {
 // go to the keys-as-rows decode kernel (dtc), other tokens to 128-row query
 // tiles (tc); without it, MHA decodes go to the CUDA-core decode kernel and
 // the rest to the general path.
-// slots: CTAs the persistent kernels run with (for the long-tile split).
+// slots: CTAs the query-tile kernel runs with (for the long-tile split).
 void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& ctx_lens,
                 int n_kv_heads, int g, int head_dim, int window, bool use_tc, int slots, Plan* out);
 
