@@ -111,12 +111,18 @@ def algorithmic_work(w):
 
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, from one ncu capture
-# of the kernel on the headline batch (compact pool); None once the kernel has
-# changed since that capture. Summaries with the commands are in profiles/.
+# of the kernel on that config's batch with the block pool sized to what the
+# batch uses (same kernel, same bytes); keyed by config, then kernel. Absent
+# (null in the line) where no capture was taken or the kernel has changed
+# since. Summaries with the commands are in profiles/.
 NCU_TRAFFIC = {
-    "decode": None,
-    "tc": None,
+    2: {"decode": 1264564480, "tc": 52505856},
+    5: {"tc": 1111393024},
 }
+
+
+def ncu_traffic(config, kernel):
+    return NCU_TRAFFIC.get(config, {}).get(kernel)
 
 
 def load_peaks():
@@ -254,13 +260,19 @@ def blas_threads():
         return len(os.sched_getaffinity(0))
 
 
-def cpu_baseline(w):
-    sub = oracle_sample(w, max_chunk_rows=768)
+def cpu_baseline(w, max_chunk_rows=4096):
+    """The oracle over the measured batch (prompt chunks cut at max_chunk_rows
+    tokens; the headline batch's 2017-token chunk is taken whole, about 10 s
+    of host work)."""
+    sub = oracle_sample(w, max_chunk_rows=max_chunk_rows)
     t = time_oracle(sub, reps=1)[0]
+    whole = int(sub.n_tokens) == int(w.n_tokens)
+    what = (f"the whole batch ({sub.n_tokens} tokens: {int((w.q_lens == 1).sum())} decodes + the prompt chunks)"
+            if whole else
+            f"{sub.n_tokens} tokens: all {int((w.q_lens == 1).sum())} decodes + first "
+            f"{int(sub.q_lens.max())} tokens of each prompt chunk")
     return {"value": sub.n_tokens / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{sub.n_tokens} tokens: all {int((w.q_lens == 1).sum())} decodes + first "
-                      f"{int(sub.q_lens.max())} tokens of each prompt chunk, float64 numpy, "
-                      f"{t:.2f} s"}
+            "sample": f"{what}, float64 numpy, {t:.2f} s"}
 
 
 def run_reference(args, w, rank, ws):
@@ -353,16 +365,24 @@ def run_fg(args, w, rank, ws, local_rank):
     # the sampler thread is started before the barrier, and every step
     # (the first included) is preceded by the L2 flush, so the device has
     # queued work while the host enqueues a step, as it does between steps
+    # a short interpreter switch interval lets the sampler thread run every
+    # couple of milliseconds while the main thread enqueues
+    switch = sys.getswitchinterval()
+    sys.setswitchinterval(2e-4)
     with ClockSampler(local_rank) as clocks:
         barrier()
         torch.cuda.synchronize()
         for i in range(args.steps):
-            flush_l2()
+            # before the first step the flush is repeated, so that the host
+            # has its first batch put done when the device gets to the step
+            for _ in range(4 if i == 0 else 1):
+                flush_l2()
             t0 = time.perf_counter()
             step(evs[i])
             host_s += time.perf_counter() - t0
         torch.cuda.synchronize()
         barrier()
+    sys.setswitchinterval(switch)
     lib_host = {k_: v_ / args.steps for k_, v_ in batch.host_profile_us(reset=True).items()}
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
     put_ms = sum(e[0].elapsed_time(e[3]) for e in evs) / len(evs)
@@ -427,16 +447,16 @@ def run_fg(args, w, rank, ws, local_rank):
         achieved = work["decode_bytes"] / (kernel_ms["decode"] / 1000) / 1e9
         roof = {"kernel": "decode (attn_decode_tc_kernel at d=128, attn_decode_kernel at d=64)", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": NCU_TRAFFIC["decode"], "algorithmic_bytes": work["decode_bytes"]}
+                "traffic": ncu_traffic(args.config, "decode"), "algorithmic_bytes": work["decode_bytes"]}
     elif work["tc_flops"] / (tf * 1e12) >= work["tc_bytes"] / (hbm * 1e9):
         achieved = work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12
         roof = {"kernel": "attn_tc_kernel (tcgen05 tiles)", "bound": "tensor", "achieved": achieved,
-                "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf, "traffic": NCU_TRAFFIC["tc"],
+                "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf, "traffic": ncu_traffic(args.config, "tc"),
                 "algorithmic_flops": work["tc_flops"]}
     else:  # its tiles are mostly grouped-query decodes: bound by the K/V bytes
         achieved = work["tc_bytes"] / (kernel_ms["tc"] / 1000) / 1e9
         roof = {"kernel": "attn_tc_kernel (tcgen05 tiles)", "bound": "hbm", "achieved": achieved,
-                "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": NCU_TRAFFIC["tc"],
+                "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": ncu_traffic(args.config, "tc"),
                 "algorithmic_bytes": work["tc_bytes"]}
     roof.update({"peak_source": f"{src} (MEASURED_PEAKS.json)" if src == "measured" else src,
                  "kernel_ms": kernel_ms,
