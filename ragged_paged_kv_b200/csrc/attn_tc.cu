@@ -520,7 +520,9 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         if (lane == 0) ptx::mbar_arrive(p_full(qt, sb));
       }
       if (!ok) break;
-      // epilogue: wait for the unit's last PV, normalise, store, free O
+      // epilogue: wait for the unit's last PV, read the O row out of TMEM
+      // half at a time (one wait per half), normalise and store it, and free
+      // O (the next unit's first P.V may start; the stores are in flight)
       const int last = lt - 1;
       if (!wait_or_flag(pv_done(qt, last & 1), (last >> 1) & 1, err, ok)) break;
       ptx::tc_fence_after();
@@ -529,15 +531,18 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         const int qh = x.h * g + (rr % g);
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          ptx::tmem_ld32(tmem + lane_base + col_o + c * 32, o);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t o[D / 2];
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            ptx::tmem_ld32(tmem + lane_base + col_o + hh * (D / 2) + c * 32,
+                           *reinterpret_cast<uint32_t(*)[32]>(&o[c * 32]));
           ptx::tmem_ld_wait();
           if (!row_ok) continue;
           if (x.part < 0) {
-            uint4* dst = reinterpret_cast<uint4*>(a.out + ((int64_t)row * a.Hq + qh) * D + c * 32);
+            uint4* dst = reinterpret_cast<uint4*>(a.out + ((int64_t)row * a.Hq + qh) * D + hh * (D / 2));
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q4 = 0; q4 < D / 16; ++q4) {
               uint32_t w[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -548,9 +553,9 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
               dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(a.part_o + (int64_t)(x.part + rr) * D + c * 32);
+            float4* dst = reinterpret_cast<float4*>(a.part_o + (int64_t)(x.part + rr) * D + hh * (D / 2));
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
+            for (int q4 = 0; q4 < D / 8; ++q4)
               dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
                                     __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
           }
