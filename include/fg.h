@@ -145,6 +145,18 @@ fg_status fg_rotary_kv_append(fg_kv_cache* cache, const fg_ragged_batch* batch, 
                               const void* k, const void* v, void* q_rot, int32_t n_q_heads,
                               double rope_theta, void* stream);
 
+/* Step 2 alone, for model families without rotary position embedding: the
+ * pages name OPT beside LLaMA and Mistral (Key points), and OPT adds learned
+ * absolute position embeddings to the hidden states before the Q/K/V
+ * projections, so its K and V enter the cache as they are. k and v: device
+ * [T][Hkv][d], 16-byte aligned; both are bit-copied to slot p % B of block
+ * block_table[s][p / B] (no other cache word changes), and the attention
+ * then takes the queries themselves as q_rot. Asynchronous on `stream`;
+ * errors as fg_rotary_kv_append (FG_ERR_INVALID_ARG for NULL or misaligned
+ * tensors, a batch whose cache is not `cache`). */
+fg_status fg_kv_append(fg_kv_cache* cache, const fg_ragged_batch* batch, const void* k, const void* v,
+                       void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Step 3: one ragged causal attention over every sequence's cached context  */
 /* ------------------------------------------------------------------------ */

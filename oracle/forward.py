@@ -9,12 +9,18 @@ from .rotary import rotate_half
 
 
 def splitfuse_pass(cache: PagedCache, block_tables, q_lens, ctx_lens, q_bits, k_bits, v_bits,
-                   theta, scale, window=0, tokens=None):
+                   theta, scale, window=0, tokens=None, rotary=True):
     """Returns (q_rot bits [T,Hq,d], k_rot bits [T,Hkv,d], O float64 [T,Hq,d]).
-    Mutates ``cache`` by the append."""
+    Mutates ``cache`` by the append. rotary=False is the pass of a family
+    without rotary embedding (OPT, named beside LLaMA and Mistral in the
+    card's Key points; its positions are learned and added before the Q/K/V
+    projections): Q and K are used as they are."""
     _, pos = token_positions(q_lens, ctx_lens)
-    q_rot = rotate_half(q_bits, pos, theta)
-    k_rot = rotate_half(k_bits, pos, theta)
+    if rotary:
+        q_rot = rotate_half(q_bits, pos, theta)
+        k_rot = rotate_half(k_bits, pos, theta)
+    else:
+        q_rot, k_rot = q_bits.copy(), k_bits.copy()
     append_kv(cache, block_tables, q_lens, ctx_lens, k_rot, v_bits)
     out = ragged_attention(cache, block_tables, q_lens, ctx_lens, q_rot, scale, window, tokens)
     return q_rot, k_rot, out

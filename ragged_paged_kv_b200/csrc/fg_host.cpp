@@ -563,8 +563,22 @@ extern "C" fg_status fg_rotary_kv_append(fg_kv_cache* c, const fg_ragged_batch* 
   cudaError_t e = fg::launch_rotary_append(
       cache_view(c), b->view, static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-      static_cast<__nv_bfloat16*>(q_rot), c->rope, n_q_heads, static_cast<cudaStream_t>(stream));
+      static_cast<__nv_bfloat16*>(q_rot), c->rope, n_q_heads, true, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "rotary_append launch");
+  return FG_OK;
+}
+
+extern "C" fg_status fg_kv_append(fg_kv_cache* c, const fg_ragged_batch* b, const void* k, const void* v,
+                                  void* stream) {
+  fg_status st = check_pass(c, b, c ? c->n_kv_heads : 1);
+  if (st) return st;
+  if (b->n_tokens == 0) return FG_OK;
+  if (!k || !v) return fail(FG_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(k) || !aligned16(v)) return fail(FG_ERR_INVALID_ARG, "k and v must be 16-byte aligned");
+  cudaError_t e = fg::launch_rotary_append(cache_view(c), b->view, nullptr, static_cast<const __nv_bfloat16*>(k),
+                                           static_cast<const __nv_bfloat16*>(v), nullptr, nullptr, 0, false,
+                                           static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
   return FG_OK;
 }
 

@@ -68,7 +68,7 @@ __host__ __device__ inline int64_t cache_offset(const CacheView& c, int64_t blk,
 cudaError_t launch_rotary_append(const CacheView& cache, const BatchView& batch,
                                  const __nv_bfloat16* q, const __nv_bfloat16* k,
                                  const __nv_bfloat16* v, __nv_bfloat16* q_rot, const double2* rope,
-                                 int n_q_heads, cudaStream_t stream);
+                                 int n_q_heads, bool rotate, cudaStream_t stream);
 
 cudaError_t launch_attention_general(const CacheView& cache, const BatchView& batch,
                                      const WorkItem* items, int n_items,

@@ -108,7 +108,9 @@ struct RotCfg {
 // memory and store 16-byte vectors, then free the stage. With three stages
 // the producer's dependent metadata loads and the copies stay ahead of the
 // arithmetic.
-template <int D>
+// ROT = false: the append alone (models without rotary embedding): the head
+// list is k | v (Hq = 0) and K is copied like V.
+template <int D, bool ROT>
 __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_kernel(
     CacheView cache, BatchView batch, const __nv_bfloat16* q, const __nv_bfloat16* k,
     const __nv_bfloat16* v, __nv_bfloat16* q_rot, const double2* __restrict__ rope, int Hq, int chunks) {
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
       m.blk = batch.bt[batch.bt_off[s] + lb];
       m.slot = pos - lb * cache.block_size;
       *reinterpret_cast<UnitMeta*>(stage + C::kMeta) = m;
-      const bool rot = h0 < Hq + Hkv;
+      const bool rot = ROT && h0 < Hq + Hkv;
       ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((h1 - h0) * ROW + (rot ? HALF * 16 : 0)));
       if (rot) ptx::bulk_g2s(stage + C::kRope, rope + (int64_t)pos * HALF, HALF * 16, &full[st]);
       // [h0, h1) cut by the q, k and v ranges of the concatenated head list
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
     const UnitMeta m = *reinterpret_cast<const UnitMeta*>(stage + C::kMeta);
     const bool blk_ok = m.blk >= 0 && m.blk < cache.n_blocks;
     if (!blk_ok && threadIdx.x == 0) atomicOr(batch.err, kErrBadBlock);
-    const int n_rot = max(0, min(m.h1, Hq + Hkv) - m.h0);  // rotated heads in this unit
+    const int n_rot = ROT ? max(0, min(m.h1, Hq + Hkv) - m.h0) : 0;  // rotated heads in this unit
     if (n_rot > 0) {
       // the rotary row is stored pair 8 g + e at entry e * GROUPS + g, so
       // these loads are conflict-free
@@ -252,14 +254,16 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
       }
     }
     if (blk_ok) {
-      // V heads of the unit: a plain copy into the cache slots
+      // V heads (and, without rotary, K heads) of the unit: a plain copy
+      // into the cache slots
       constexpr int VCH = D / 8;  // 16-byte pieces per head
-      const int v0 = max(m.h0, Hq + Hkv);
+      const int v0 = ROT ? max(m.h0, Hq + Hkv) : m.h0;
       const int nv = max(0, m.h1 - v0) * VCH;
       for (int ci = threadIdx.x; ci < nv; ci += kConsumers) {
         const int hl = ci / VCH, c = ci - hl * VCH;
-        const int h = v0 + hl - Hq - Hkv;
-        *reinterpret_cast<uint4*>(cache.base + cache_offset(cache, m.blk, 1, h, m.slot) + c * 8) =
+        const int hk = v0 + hl - Hq;  // index in the k | v head list
+        const int kv = hk >= Hkv ? 1 : 0;
+        *reinterpret_cast<uint4*>(cache.base + cache_offset(cache, m.blk, kv, hk - kv * Hkv, m.slot) + c * 8) =
             *reinterpret_cast<const uint4*>(stage + (v0 - m.h0 + hl) * ROW + c * 16);
       }
     }
@@ -274,8 +278,9 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
 cudaError_t launch_rotary_append(const CacheView& cache, const BatchView& batch,
                                  const __nv_bfloat16* q, const __nv_bfloat16* k,
                                  const __nv_bfloat16* v, __nv_bfloat16* q_rot, const double2* rope,
-                                 int n_q_heads, cudaStream_t stream) {
+                                 int n_q_heads, bool rotate, cudaStream_t stream) {
   if (batch.n_tokens == 0) return cudaSuccess;
+  if (!rotate) n_q_heads = 0;
   const int chunks = (n_q_heads + 2 * cache.n_kv_heads + kChunkHeads - 1) / kChunkHeads;
   const int64_t units = (int64_t)batch.n_tokens * chunks;
   if (units > (int64_t)1 << 30) return cudaErrorInvalidConfiguration;
@@ -283,12 +288,21 @@ cudaError_t launch_rotary_append(const CacheView& cache, const BatchView& batch,
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     sms = 148;
   const int grid = (int)std::min<int64_t>(units, (int64_t)sms * kCtasPerSm);
-  if (cache.head_dim == 128)
-    rotary_append_kernel<128><<<grid, kConsumers + 32, RotCfg<128>::kSmem, stream>>>(
-        cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
-  else
-    rotary_append_kernel<64><<<grid, kConsumers + 32, RotCfg<64>::kSmem, stream>>>(
-        cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
+  if (cache.head_dim == 128) {
+    if (rotate)
+      rotary_append_kernel<128, true><<<grid, kConsumers + 32, RotCfg<128>::kSmem, stream>>>(
+          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
+    else
+      rotary_append_kernel<128, false><<<grid, kConsumers + 32, RotCfg<128>::kSmem, stream>>>(
+          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
+  } else {
+    if (rotate)
+      rotary_append_kernel<64, true><<<grid, kConsumers + 32, RotCfg<64>::kSmem, stream>>>(
+          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
+    else
+      rotary_append_kernel<64, false><<<grid, kConsumers + 32, RotCfg<64>::kSmem, stream>>>(
+          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
+  }
   return cudaGetLastError();
 }
 

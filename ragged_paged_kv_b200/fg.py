@@ -49,6 +49,7 @@ def lib() -> ctypes.CDLL:
         "fg_ragged_batch_shape": [V, _c_int32_p, _c_int32_p],
         "fg_ragged_batch_destroy": [V],
         "fg_rotary_kv_append": [V, V, V, V, V, V, I32, D, V],
+        "fg_kv_append": [V, V, V, V, V],
         "fg_ragged_attention": [V, V, V, V, I32, F, I32, V],
         "fg_ragged_attention_noalloc": [V, V, V, V, I32, F, I32, V],
         "fg_device_status": [V, V],
@@ -246,6 +247,13 @@ def rotary_kv_append(cache: KVCache, batch: RaggedBatch, q, k, v, q_rot, n_q_hea
                                      _dev_ptr(v, "v"), _dev_ptr(q_rot, "q_rot"), int(n_q_heads),
                                      float(rope_theta), _stream_ptr(stream)),
            "fg_rotary_kv_append")
+
+
+def kv_append(cache: KVCache, batch: RaggedBatch, k, v, stream=None):
+    """Append without rotary (learned-position families such as OPT): K and V
+    go into the cache unchanged; pass q itself as q_rot to the attention."""
+    _check(lib().fg_kv_append(cache.handle, batch.handle, _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                              _stream_ptr(stream)), "fg_kv_append")
 
 
 def ragged_attention(cache: KVCache, batch: RaggedBatch, q_rot, out, n_q_heads: int,

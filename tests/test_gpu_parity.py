@@ -53,7 +53,7 @@ def run_gpu(w, keep, cache=None, fill=True, write_ctx=True, inplace=False, other
     return cache, batch, q_rot, out, kept
 
 
-def run_oracle(w, kept, tokens=None, pc=None):
+def run_oracle(w, kept, tokens=None, pc=None, rotary=True):
     if pc is None:
         pc = PagedCache(w.n_blocks, w.n_kv_heads, w.block_size, w.head_dim, fill=SENTINEL)
         for s, (ids, blocks) in kept.items():
@@ -61,7 +61,7 @@ def run_oracle(w, kept, tokens=None, pc=None):
                 pc.blocks[int(b)] = blocks[i].copy()
     q, k, v = w.qkv()
     q_rot, _, out = splitfuse_pass(pc, w.block_tables, w.q_lens, w.ctx_lens, q, k, v,
-                                   w.rope_theta, w.softmax_scale, w.sliding_window, tokens)
+                                   w.rope_theta, w.softmax_scale, w.sliding_window, tokens, rotary=rotary)
     return pc, q_rot, out
 
 
@@ -266,3 +266,31 @@ def test_overlapped_schedule_gives_bit_identical_output():
             outs.append(to_bits(out))
             _free(cache, batch)
         assert np.array_equal(outs[0], outs[1]), w.name
+
+
+@pytest.mark.parametrize("which", ["tiny", "gqa_d128"])
+def test_append_without_rotary(which):
+    """fg_kv_append (families without rotary embedding, such as OPT): every
+    word of the sequences' cache blocks bit-exact, and the attention over q
+    itself within tolerance of the oracle's no-rotary pass."""
+    w = W.config1() if which == "tiny" else W._make("no_rotary_gqa", 8, 2, 128, 64, [0, 1, 2], [300, 1, 17],
+                                                      [0, 700, 70], seed=9, budget=318)
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+    fixtures.fill(cache.tensor)
+    kept = fixtures.write_context(w, cache.tensor, set(range(w.n_seqs)))
+    batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+    batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables)
+    q, k, v = fixtures.qkv_device(w)
+    out = torch.full_like(q, float("nan"))
+    fg.kv_append(cache, batch, k, v)
+    fg.ragged_attention(cache, batch, q, out, w.n_q_heads, w.softmax_scale, w.sliding_window)
+    torch.cuda.synchronize()
+    batch.device_status()
+    pc, q_ref, ref = run_oracle(w, kept, rotary=False)
+    for s in range(w.n_seqs):
+        ids = w.block_tables[s, :w.blocks_used(s)].astype(np.int64)
+        dev = to_bits(cache.tensor[torch.from_numpy(ids).cuda()])
+        for i, b in enumerate(ids):
+            assert np.array_equal(dev[i], pc.block(int(b))), f"cache block {b} of seq {s} differs"
+    assert_close(bf16_to_f64(to_bits(out)), ref, w.name)
+    _free(cache, batch)

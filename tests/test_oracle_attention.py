@@ -193,3 +193,35 @@ def test_sampled_rows_equal_full_rows():
     s = ragged_attention(c, w.block_tables, w.q_lens, w.ctx_lens, qr, w.softmax_scale, 0, tok)
     assert np.abs(s[tok] - o[tok]).max() <= 1e-12
     assert np.isnan(s[1]).all()
+
+
+def test_pass_without_rotary_appends_the_bits_and_attends_with_q_itself():
+    """The no-rotary pass (learned-position families): the cache receives K and
+    V bit for bit, Q is not changed, and the attention equals brute force on
+    the unrotated Q and K."""
+    from oracle.forward import splitfuse_pass
+    from ragged_paged_kv_b200 import workloads as W
+    w = W.config1()
+    pc = PagedCache(w.n_blocks, w.n_kv_heads, w.block_size, w.head_dim, fill=0)
+    for s, kc, vc in w.contexts():
+        pc.write_positions(w.block_tables[s], np.arange(kc.shape[0]), kc, vc)
+    q, k, v = w.qkv()
+    q_rot, k_rot, out = splitfuse_pass(pc, w.block_tables, w.q_lens, w.ctx_lens, q, k, v, w.rope_theta,
+                                       w.softmax_scale, rotary=False)
+    assert np.array_equal(q_rot, q) and np.array_equal(k_rot, k)
+    cu = np.concatenate([[0], np.cumsum(w.q_lens)])
+    for s in range(w.n_seqs):
+        L = int(w.ctx_lens[s] + w.q_lens[s])
+        Kc, Vc = pc.gather(w.block_tables[s], L)
+        assert np.array_equal(Kc[w.ctx_lens[s]:], k[cu[s]:cu[s + 1]])
+        assert np.array_equal(Vc[w.ctx_lens[s]:], v[cu[s]:cu[s + 1]])
+        # brute force: explicit causal softmax over the gathered context
+        Kf, Vf = bf16_bits_to_f64(Kc), bf16_bits_to_f64(Vc)
+        for j in range(int(w.q_lens[s])):
+            p = int(w.ctx_lens[s]) + j
+            for h in range(w.n_q_heads):
+                hk = h // (w.n_q_heads // w.n_kv_heads)
+                z = w.softmax_scale * (Kf[:p + 1, hk] @ bf16_bits_to_f64(q[cu[s] + j, h]))
+                e = np.exp(z - z.max())
+                ref = (e[:, None] * Vf[:p + 1, hk]).sum(0) / e.sum()
+                assert np.allclose(out[cu[s] + j, h], ref, rtol=0, atol=1e-12)
