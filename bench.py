@@ -495,6 +495,77 @@ def run_fg(args, w, rank, ws, local_rank):
     return 0
 
 
+def sweep_workload(n_tokens, n_decodes=32, seed=11):
+    """Llama-2-7B-shape batch of n_tokens: n_decodes one-token decodes
+    (contexts ~U[512, 4096]) plus one prompt chunk of the rest at context 1024."""
+    from ragged_paged_kv_b200 import workloads as W
+    rng = np.random.default_rng(seed)
+    ctx = rng.integers(512, 4097, n_decodes).tolist()
+    q = [1] * n_decodes
+    if n_tokens > n_decodes:
+        q.append(n_tokens - n_decodes)
+        ctx.append(1024)
+    return W._make(f"sweep_{n_tokens}", 32, 32, 128, 64, list(range(len(q))), q, ctx, seed=seed,
+                   budget=int(sum(q)), note="token sweep")
+
+
+def time_step(w, steps, warmup, dev):
+    """Mean device time (ms) of put + rotary/append + attention over `steps`
+    steps after `warmup`, L2 flushed (write + read of 256 MB) before each."""
+    import torch
+    from ragged_paged_kv_b200 import fg, fixtures
+    stream = torch.cuda.Stream(device=dev)
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim, device=dev)
+    fixtures.fill(cache.tensor, 0)
+    fixtures.write_context(w, cache.tensor, keep=(), others="pool")
+    batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+    q, k, v = fixtures.qkv_device(w, dev)
+    q_rot, out = torch.empty_like(q), torch.empty_like(q)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    evs = []
+    for i in range(warmup + steps):
+        with torch.cuda.stream(stream):
+            for _ in range(4 if i == warmup else 1):
+                flush.zero_()
+                flush.sum()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, stream)
+        fg.rotary_kv_append(cache, batch, q, k, v, q_rot, w.n_q_heads, w.rope_theta, stream)
+        fg.ragged_attention(cache, batch, q_rot, out, w.n_q_heads, w.softmax_scale, w.sliding_window, stream)
+        e[1].record(stream)
+        if i >= warmup:
+            evs.append(e)
+    torch.cuda.synchronize()
+    batch.device_status(stream)
+    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    cache.close()
+    batch.close()
+    return ms
+
+
+def run_token_sweep(args):
+    """Forward latency and throughput of the attention path against the
+    tokens in a pass (the card's observation that latency follows the token
+    count and throughput saturates, and its equal-split argument from the
+    concavity of throughput): one JSON line per point, then the measured
+    total time of splitting N tokens over two passes unevenly vs evenly."""
+    import torch
+    dev = torch.device("cuda", 0)
+    pts = {}
+    for n in (64, 128, 256, 512, 1024, 2048, 3072, 3584, 4096, 6144, 8192):
+        ms = time_step(sweep_workload(n), args.steps, args.warmup, dev)
+        pts[n] = ms
+        print(json.dumps({"kind": "token_sweep", "tokens": n, "decodes": 32, "prefill_tokens": max(0, n - 32),
+                          "ms_per_pass": ms, "tokens_per_s": n / ms * 1e3}), flush=True)
+    for total, parts in ((4096, ((2048, 2048), (1024, 3072), (512, 3584))),
+                         (8192, ((4096, 4096), (2048, 6144)))):
+        for a, b in parts:
+            print(json.dumps({"kind": "split_check", "total_tokens": total, "passes": [a, b],
+                              "ms_total": pts[a] + pts[b]}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -507,9 +578,13 @@ def main():
                     help="run the query-tile kernel beside the decode kernel on a second stream")
     ap.add_argument("--compact-pool", action="store_true",
                     help="size the block pool to what the batch uses (small ncu captures)")
+    ap.add_argument("--sweep-tokens", action="store_true",
+                    help="latency/throughput against tokens per pass (one GPU; JSON lines, no contract line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.sweep_tokens:
+        return run_token_sweep(args)
     from ragged_paged_kv_b200 import workloads as W
     if args.config == 3 and args.impl == "fg":
         import torch
