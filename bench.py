@@ -566,6 +566,49 @@ def run_token_sweep(args):
     return 0
 
 
+def run_qkv_fused(args, w):
+    """The Q/K/V projection fused with rotary + append on the headline batch's
+    tokens at Llama-2-7B width (hidden 4096, 96 heads of 128 out): one JSON
+    line with its device time, TFLOP/s and fraction of the measured bf16
+    peak (kind "qkv_fused", not the contract line)."""
+    import torch
+    from ragged_paged_kv_b200 import fg, fixtures
+    dev = torch.device("cuda", 0)
+    hidden = 4096
+    stream = torch.cuda.Stream(device=dev)
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim, device=dev)
+    fixtures.fill(cache.tensor, 0)
+    fixtures.write_context(w, cache.tensor, keep=(), others="pool")
+    batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+    g = torch.Generator(device=dev).manual_seed(7)
+    x = torch.randn((w.n_tokens, hidden), generator=g, device=dev).to(torch.bfloat16)
+    n_out = (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim
+    wq = (torch.randn((n_out, hidden), generator=g, device=dev) / hidden ** 0.5).to(torch.bfloat16)
+    q_rot = torch.empty((w.n_tokens, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, stream)
+    evs = []
+    for i in range(args.warmup + args.steps):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            flush.sum()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        fg.qkv_rotary_kv_append(cache, batch, x, wq, q_rot, w.n_q_heads, w.rope_theta, stream)
+        e[1].record(stream)
+        if i >= args.warmup:
+            evs.append(e)
+    torch.cuda.synchronize()
+    batch.device_status(stream)
+    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    flops = 2.0 * w.n_tokens * hidden * n_out
+    hbm, tf, src = load_peaks()
+    print(json.dumps({"kind": "qkv_fused", "workload": f"{w.name}: T={w.n_tokens}, hidden={hidden}, out={n_out}",
+                      "ms": ms, "tflops": flops / ms / 1e9, "peak_tflops": tf, "frac": flops / ms / 1e9 / tf,
+                      "peak_source": src}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -578,6 +621,8 @@ def main():
                     help="run the query-tile kernel beside the decode kernel on a second stream")
     ap.add_argument("--compact-pool", action="store_true",
                     help="size the block pool to what the batch uses (small ncu captures)")
+    ap.add_argument("--qkv-fused", action="store_true",
+                    help="time the fused Q/K/V projection + rotary + append (one GPU; JSON line, no contract line)")
     ap.add_argument("--sweep-tokens", action="store_true",
                     help="latency/throughput against tokens per pass (one GPU; JSON lines, no contract line)")
     args = ap.parse_args()
@@ -597,6 +642,8 @@ def main():
         w = W._make(w.name, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.seq_ids,
                     w.q_lens, w.ctx_lens, w.seed, w.budget, n_blocks=need + 16,
                     window=w.sliding_window, note=w.note + "; compact pool")
+    if args.qkv_fused:
+        return run_qkv_fused(args, w)
     if args.impl == "reference":
         rank, ws = init_dist("gloo")
         rc = run_reference(args, w, rank, ws)

@@ -145,6 +145,24 @@ fg_status fg_rotary_kv_append(fg_kv_cache* cache, const fg_ragged_batch* batch, 
                               const void* k, const void* v, void* q_rot, int32_t n_q_heads,
                               double rope_theta, void* stream);
 
+/* The Q/K/V projection fused with steps 1 and 2 (the GEMM that produces q,
+ * k and v for this hot path, kept on the device): qkv = x w_qkv^T with x
+ * device [T][hidden] bf16 (T = the batch's tokens) and w_qkv device
+ * [(n_q_heads + 2 Hkv) d][hidden] bf16 (rows: the q heads, then k, then v,
+ * d rows each; the layout of a linear layer's weight), fp32 accumulation;
+ * each output is rounded once to bf16, as a projection with bf16 output
+ * would, then q and k are rotated and stored exactly as
+ * fg_rotary_kv_append does (q_rot device [T][n_q_heads][d]; K_rot and V
+ * bit-copied into slot p % B of block block_table[s][p / B]). hidden must be
+ * a positive multiple of 64; x, w_qkv and q_rot 16-byte aligned. The result
+ * equals the projection followed by fg_rotary_kv_append up to the
+ * projection's own rounding (fp32 sums in another order can round a value to
+ * the neighbouring bf16). Asynchronous on `stream`; the first call for a
+ * rope_theta and position range builds the cos/sin table (synchronous). */
+fg_status fg_qkv_rotary_kv_append(fg_kv_cache* cache, const fg_ragged_batch* batch, const void* x,
+                                  const void* w_qkv, int32_t hidden, void* q_rot, int32_t n_q_heads,
+                                  double rope_theta, void* stream);
+
 /* Step 2 alone, for model families without rotary position embedding: the
  * pages name OPT beside LLaMA and Mistral (Key points), and OPT adds learned
  * absolute position embeddings to the hidden states before the Q/K/V

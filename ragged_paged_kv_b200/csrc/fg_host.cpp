@@ -1041,5 +1041,46 @@ fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, co
   return FG_OK;
 }
 
+// 2-D bf16 view (inner dim `inner`, outer dim `outer`, row stride inner * 2 B)
+// with boxes of 64 x box_rows, 128-byte swizzle: the K-major operand layout
+// of the projection's MMAs.
+static bool make_rows_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+extern "C" fg_status fg_qkv_rotary_kv_append(fg_kv_cache* c, const fg_ragged_batch* b, const void* x,
+                                             const void* w_qkv, int32_t hidden, void* q_rot, int32_t n_q_heads,
+                                             double rope_theta, void* stream) {
+  fg_status st = check_pass(c, b, n_q_heads);
+  if (st) return st;
+  if (!(rope_theta > 0.0)) return fail(FG_ERR_INVALID_ARG, "rope_theta must be > 0");
+  if (hidden < 64 || hidden % 64) return fail(FG_ERR_UNSUPPORTED, "hidden %d is not a positive multiple of 64", hidden);
+  if (b->n_tokens == 0) return FG_OK;
+  if (!x || !w_qkv || !q_rot) return fail(FG_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q_rot))
+    return fail(FG_ERR_INVALID_ARG, "x, w_qkv and q_rot must be 16-byte aligned");
+  st = ensure_rope(c, rope_theta, b->max_pos);
+  if (st) return st;
+  const int d = c->head_dim;
+  const uint64_t n_out = (uint64_t)(n_q_heads + 2 * c->n_kv_heads) * d;
+  CUtensorMap tm_x, tm_w;
+  if (!make_rows_map(&tm_x, x, (uint64_t)hidden, (uint64_t)b->n_tokens, 128) ||
+      !make_rows_map(&tm_w, w_qkv, (uint64_t)hidden, n_out, (uint32_t)d))
+    return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for x or w_qkv");
+  cudaError_t e = fg::launch_qkv_rotary_append(&tm_x, &tm_w, cache_view(c), b->view,
+                                               static_cast<__nv_bfloat16*>(q_rot), c->rope, n_q_heads, hidden,
+                                               static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qkv_rotary_append launch");
+  return FG_OK;
+}
+
 // Sets the thread-local error text (for entry points defined in other files).
 fg_status fg_set_error(fg_status st, const char* msg) { return fail(st, "%s", msg); }

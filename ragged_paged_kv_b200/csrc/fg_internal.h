@@ -100,6 +100,10 @@ cudaError_t launch_attention_decode_tc(const void* tm_q1, const void* tm_kv, con
                                        int sm_tc_end, const int* tc_counter, int n_tc, bool pdl,
                                        cudaStream_t stream);
 
+cudaError_t launch_qkv_rotary_append(const void* tm_x, const void* tm_w, const CacheView& cache,
+                                     const BatchView& batch, __nv_bfloat16* q_rot, const double2* rope,
+                                     int n_q_heads, int hidden, cudaStream_t stream);
+
 cudaError_t launch_combine(const BatchView& batch, const CombineItem* items, int n_items,
                            int max_rows, const float* part_o, const float* part_ml,
                            __nv_bfloat16* out, int n_q_heads, int g, int head_dim, bool pdl,

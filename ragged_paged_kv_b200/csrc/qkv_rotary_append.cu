@@ -1,0 +1,236 @@
+// The Q/K/V projection fused with steps 1 and 2: qkv = x W^T on the tensor
+// cores (tcgen05, fp32 accumulation in TMEM), and in the epilogue every
+// output row is rounded to bf16 (as a projection with bf16 output would), Q
+// and K rotated exactly as fg_rotary_kv_append does, Q written to q_rot and
+// K, V written into their cache slots. The projected Q/K/V never make a round
+// trip through HBM.
+//
+// A CTA computes one tile: 128 tokens x one head (d output features), so the
+// epilogue thread that owns a token holds the head's whole row, both halves
+// of every rotary pair. Roles: warp 0 (one thread) streams 64-wide K slices
+// of x and W with 2-D TMA boxes (128-byte swizzle) into a 3-stage ring, warp
+// 1 (one thread) issues the MMAs, warps 2-5 (TMEM lanes 32 (w % 4) ..) run
+// the epilogue. Every wait is bounded.
+#include <cuda.h>
+
+#include <cfloat>
+
+#include "fg_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace fg {
+namespace {
+
+constexpr long long kWaitLimit = 1LL << 31;
+
+template <int D>
+struct QkvCfg {
+  static constexpr int BM = 128;  // tokens per tile
+  static constexpr int BK = 64;   // hidden features per stage (one 128-byte row)
+  static constexpr int ST = 3;
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = D * BK * 2;
+  static constexpr int kStage = kABytes + kBBytes;
+  static constexpr int kOffBar = ST * kStage;
+  static constexpr int kNumBars = 2 * ST + 1;  // full[ST], empty[ST], acc_full
+  static constexpr int kSmem = kOffBar + kNumBars * 8 + 16;
+  static constexpr int kThreads = 192;
+  static constexpr uint32_t kTmemCols = D < 32 ? 32 : D;
+};
+
+struct QkvArgs {
+  CacheView cache;
+  BatchView batch;
+  __nv_bfloat16* q_rot;
+  const double2* rope;  // the rotary table, see below
+  int Hq;
+  int hidden;
+};
+
+// float64 -> bf16 with one rounding (truncate to float, force the last bit on
+// when anything was dropped: round to odd, then round to nearest even).
+__device__ __forceinline__ unsigned short f64_to_bf16(double x) {
+  float f = __double2float_rz(x);
+  if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int32_t* err, bool& ok) {
+  if (!ok) return false;
+  if (!ptx::mbar_wait_bounded(bar, parity, kWaitLimit)) {
+    atomicOr(err, kErrTimeout);
+    ok = false;
+  }
+  return ok;
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 2) qkv_rotary_append_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                                  const __grid_constant__ CUtensorMap tm_w,
+                                                                  QkvArgs a) {
+  using C = QkvCfg<D>;
+  constexpr int HALF = D / 2;
+  constexpr int GROUPS = HALF / 8;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  if (ptx::smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(a.batch.err, kErrBadIndex);
+    return;
+  }
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + C::ST;
+  uint64_t* acc_full = empty + C::ST;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * C::BM;  // first token of the tile
+  const int head = blockIdx.y;        // in the q | k | v head list
+  const int n_k = a.hidden / C::BK;
+  int32_t* err = a.batch.err;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::ST; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], 1);
+    }
+    ptx::mbar_init(acc_full, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- loads
+    if (lane == 0) {
+      for (int i = 0; i < n_k && ok; ++i) {
+        const int st = i % C::ST;
+        if (i >= C::ST && !wait_or_flag(&empty[st], ((i / C::ST) - 1) & 1, err, ok)) break;
+        ptx::mbar_arrive_expect_tx(&full[st], C::kStage);
+        unsigned char* s = smem + st * C::kStage;
+        ptx::tma_load_2d(s, &tm_x, i * C::BK, t0, &full[st]);  // rows past T read as zeros
+        ptx::tma_load_2d(s + C::kABytes, &tm_w, i * C::BK, head * D, &full[st]);
+      }
+      for (int i = max(0, n_k - C::ST); i < n_k && ok; ++i)
+        wait_or_flag(&full[i % C::ST], (i / C::ST) & 1, err, ok);
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(C::BM, D, 0, 0);
+      const uint32_t base = ptx::smem_u32(smem);
+      for (int i = 0; i < n_k && ok; ++i) {
+        const int st = i % C::ST;
+        if (!wait_or_flag(&full[st], (i / C::ST) & 1, err, ok)) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk) {
+          const uint64_t ad = ptx::smem_desc_sw128(base + st * C::kStage + kk * 32, 16, 1024);
+          const uint64_t bd = ptx::smem_desc_sw128(base + st * C::kStage + C::kABytes + kk * 32, 16, 1024);
+          ptx::mma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(&empty[st]);
+      }
+      ptx::mma_commit(acc_full);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int r = (warp & 3) * 32 + lane;  // token row == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int t = t0 + r;
+    const bool live = (warp & 3) * 32 + t0 < a.batch.n_tokens;
+    if (wait_or_flag(acc_full, 0, err, ok) && live) {
+      ptx::tc_fence_after();
+      uint32_t acc[D];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c)
+        ptx::tmem_ld32(tmem + lane_base + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[c * 32]));
+      ptx::tmem_ld_wait();
+      if (t < a.batch.n_tokens) {
+        // the projection's bf16 output, in place (bits in the low half)
+#pragma unroll
+        for (int e = 0; e < D; ++e) acc[e] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(acc[e])));
+        const int Hkv = a.cache.n_kv_heads;
+        const int s = a.batch.tok_seq[t];
+        const int p = a.batch.ctx[s] + (t - a.batch.cu_q[s]);
+        __nv_bfloat16* dst = nullptr;
+        if (head < a.Hq) {
+          dst = a.q_rot + ((int64_t)t * a.Hq + head) * D;
+        } else {
+          const int lb = p / a.cache.block_size;
+          const int32_t blk = a.batch.bt[a.batch.bt_off[s] + lb];
+          if (blk >= 0 && blk < a.cache.n_blocks) {
+            const int kv = head < a.Hq + Hkv ? 0 : 1;
+            dst = a.cache.base +
+                  cache_offset(a.cache, blk, kv, head - a.Hq - kv * Hkv, p - lb * a.cache.block_size);
+          } else {
+            atomicOr(err, kErrBadBlock);
+          }
+        }
+        if (head < a.Hq + Hkv) {
+          // rotate-half in double, one rounding to bf16; the table row of
+          // position p holds pair i = 8 g + e at entry e * GROUPS + g, times
+          // 2^896
+          const double2* rrow = a.rope + (int64_t)p * HALF;
+#pragma unroll
+          for (int i = 0; i < HALF; ++i) {
+            const double2 cs = rrow[(i & 7) * GROUPS + (i >> 3)];
+            const double c = cs.x * 0x1p-896, sn = cs.y * 0x1p-896;
+            const double x1 = (double)__uint_as_float(acc[i] << 16);
+            const double x2 = (double)__uint_as_float(acc[i + HALF] << 16);
+            acc[i] = f64_to_bf16(__dsub_rn(__dmul_rn(x1, c), __dmul_rn(x2, sn)));
+            acc[i + HALF] = f64_to_bf16(__dadd_rn(__dmul_rn(x2, c), __dmul_rn(x1, sn)));
+          }
+        }
+        if (dst) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int q = 0; q < D / 8; ++q)
+            d4[q] = make_uint4(acc[8 * q] | (acc[8 * q + 1] << 16), acc[8 * q + 2] | (acc[8 * q + 3] << 16),
+                               acc[8 * q + 4] | (acc[8 * q + 5] << 16), acc[8 * q + 6] | (acc[8 * q + 7] << 16));
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_qkv_d(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const QkvArgs& args,
+                         int n_heads_total, cudaStream_t stream) {
+  using C = QkvCfg<D>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(qkv_rotary_append_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  dim3 grid((args.batch.n_tokens + C::BM - 1) / C::BM, n_heads_total);
+  qkv_rotary_append_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tm_x, tm_w, args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_qkv_rotary_append(const void* tm_x, const void* tm_w, const CacheView& cache,
+                                     const BatchView& batch, __nv_bfloat16* q_rot, const double2* rope,
+                                     int n_q_heads, int hidden, cudaStream_t stream) {
+  if (batch.n_tokens == 0) return cudaSuccess;
+  QkvArgs args{cache, batch, q_rot, rope, n_q_heads, hidden};
+  const int heads = n_q_heads + 2 * cache.n_kv_heads;
+  const CUtensorMap& x = *static_cast<const CUtensorMap*>(tm_x);
+  const CUtensorMap& w = *static_cast<const CUtensorMap*>(tm_w);
+  if (cache.head_dim == 128) return launch_qkv_d<128>(x, w, args, heads, stream);
+  return launch_qkv_d<64>(x, w, args, heads, stream);
+}
+
+}  // namespace fg

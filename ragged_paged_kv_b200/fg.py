@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
         "fg_ragged_batch_destroy": [V],
         "fg_rotary_kv_append": [V, V, V, V, V, V, I32, D, V],
         "fg_kv_append": [V, V, V, V, V],
+        "fg_qkv_rotary_kv_append": [V, V, V, V, I32, V, I32, D, V],
         "fg_ragged_attention": [V, V, V, V, I32, F, I32, V],
         "fg_ragged_attention_noalloc": [V, V, V, V, I32, F, I32, V],
         "fg_device_status": [V, V],
@@ -247,6 +248,18 @@ def rotary_kv_append(cache: KVCache, batch: RaggedBatch, q, k, v, q_rot, n_q_hea
                                      _dev_ptr(v, "v"), _dev_ptr(q_rot, "q_rot"), int(n_q_heads),
                                      float(rope_theta), _stream_ptr(stream)),
            "fg_rotary_kv_append")
+
+
+def qkv_rotary_kv_append(cache: KVCache, batch: RaggedBatch, x, w_qkv, q_rot, n_q_heads: int,
+                         rope_theta: float, stream=None):
+    """The Q/K/V projection x w_qkv^T fused with rotary + append (see
+    fg_qkv_rotary_kv_append): x [T, hidden], w_qkv [(Hq + 2 Hkv) d, hidden]."""
+    if x.dim() != 2 or w_qkv.dim() != 2 or x.shape[1] != w_qkv.shape[1]:
+        raise ValueError("x must be [T, hidden] and w_qkv [(Hq + 2 Hkv) d, hidden]")
+    _check(lib().fg_qkv_rotary_kv_append(cache.handle, batch.handle, _dev_ptr(x, "x"), _dev_ptr(w_qkv, "w_qkv"),
+                                         int(x.shape[1]), _dev_ptr(q_rot, "q_rot"), int(n_q_heads),
+                                         float(rope_theta), _stream_ptr(stream)),
+           "fg_qkv_rotary_kv_append")
 
 
 def kv_append(cache: KVCache, batch: RaggedBatch, k, v, stream=None):

@@ -192,7 +192,10 @@ def test_empty_batch_is_a_no_op():
 
 @pytest.mark.parametrize("B,d,Hq,Hkv,window", [
     (16, 64, 4, 4, 0), (32, 128, 8, 2, 0), (64, 128, 8, 1, 0), (128, 64, 6, 3, 0),
-    (16, 128, 16, 2, 37), (64, 64, 4, 4, 300), (128, 128, 32, 8, 0), (32, 64, 16, 16, 1)])
+    (16, 128, 16, 2, 37), (64, 64, 4, 4, 300), (128, 128, 32, 8, 0), (32, 64, 16, 16, 1),
+    # group sizes that are not powers of two (the general path), the largest
+    # grouped decode (g = 16) and a group past it (decodes as query tiles)
+    (64, 128, 12, 4, 0), (32, 64, 10, 2, 50), (64, 128, 32, 2, 0), (64, 128, 64, 2, 0)])
 def test_shape_sweep(B, d, Hq, Hkv, window):
     """Ragged tails everywhere: lengths off every tile / block / stage size."""
     rng = np.random.default_rng(B * 7 + d + Hq * 3 + Hkv + window)
@@ -292,5 +295,80 @@ def test_append_without_rotary(which):
         dev = to_bits(cache.tensor[torch.from_numpy(ids).cuda()])
         for i, b in enumerate(ids):
             assert np.array_equal(dev[i], pc.block(int(b))), f"cache block {b} of seq {s} differs"
+    assert_close(bf16_to_f64(to_bits(out)), ref, w.name)
+    _free(cache, batch)
+
+
+@pytest.mark.parametrize("which", ["mha_d64", "gqa_d128"])
+def test_fused_qkv_projection_rotary_append(which):
+    """fg_qkv_rotary_kv_append: the projection x W^T fused with rotary and the
+    append. Against the oracle's exact projection (rounded once to bf16) the
+    GPU's fp32 sums may round a value to the neighbouring bf16, so q_rot and
+    the new cache slots are checked to within two bf16 units with almost all
+    words identical, the prior context bit-exact, and the attention output to
+    the usual tolerance."""
+    from oracle import qkv_projection
+    if which == "mha_d64":
+        w = W._make("qkv_mha_d64", 4, 4, 64, 16, [0, 1, 2, 3], [40, 1, 1, 22], [0, 37, 5, 10], seed=21,
+                    budget=64)
+        hidden = 256
+    else:
+        w = W._make("qkv_gqa_d128", 8, 2, 128, 64, [0, 1, 2], [300, 1, 17], [0, 700, 70], seed=22, budget=318)
+        hidden = 512
+    rng = np.random.default_rng(23)
+    x_bits = W.f32_to_bf16_bits(rng.standard_normal((w.n_tokens, hidden)).astype(np.float32))
+    n_out = (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim
+    w_bits = W.f32_to_bf16_bits((rng.standard_normal((n_out, hidden)) / np.sqrt(hidden)).astype(np.float32))
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+    fixtures.fill(cache.tensor)
+    kept = fixtures.write_context(w, cache.tensor, set(range(w.n_seqs)))
+    batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+    batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables)
+    xd = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    wd = torch.from_numpy(w_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    q_rot = torch.empty((w.n_tokens, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device="cuda")
+    out = torch.full_like(q_rot, float("nan"))
+    fg.qkv_rotary_kv_append(cache, batch, xd, wd, q_rot, w.n_q_heads, w.rope_theta)
+    fg.ragged_attention(cache, batch, q_rot, out, w.n_q_heads, w.softmax_scale, w.sliding_window)
+    torch.cuda.synchronize()
+    batch.device_status()
+    q, k, v = qkv_projection(x_bits, w_bits, w.n_q_heads, w.n_kv_heads, w.head_dim)
+    pc = PagedCache(w.n_blocks, w.n_kv_heads, w.block_size, w.head_dim, fill=SENTINEL)
+    for s, (ids, blocks) in kept.items():
+        for i, b in enumerate(ids):
+            pc.blocks[int(b)] = blocks[i].copy()
+    q_ref, k_ref, ref = splitfuse_pass(pc, w.block_tables, w.q_lens, w.ctx_lens, q, k, v, w.rope_theta,
+                                       w.softmax_scale, w.sliding_window)
+
+    def pair_mag(pre_bits):
+        # |x_i| + |x_{i+d/2}|: a rotated value moves by at most about a bf16
+        # unit of this when its inputs are off by one unit each
+        x = np.abs(bf16_to_f64(pre_bits))
+        h = x.shape[-1] // 2
+        m = x[..., :h] + x[..., h:]
+        return np.concatenate([m, m], axis=-1)
+
+    def near(got_bits, ref_bits, scale, what):
+        g, r = bf16_to_f64(got_bits), bf16_to_f64(ref_bits)
+        assert np.all(np.abs(g - r) <= 2.0 ** -6 * (scale + np.abs(r))), f"{what}: beyond two bf16 units"
+        assert np.mean(got_bits != ref_bits) < 0.01, f"{what}: {np.mean(got_bits != ref_bits):.3%} words differ"
+
+    near(to_bits(q_rot), q_ref, pair_mag(q), "q_rot")
+    cu = np.concatenate([[0], np.cumsum(w.q_lens)])
+    for s in range(w.n_seqs):
+        ids = w.block_tables[s, :w.blocks_used(s)].astype(np.int64)
+        dev = to_bits(cache.tensor[torch.from_numpy(ids).cuda()])
+        ref_blocks = np.stack([pc.block(int(b)) for b in ids])
+        c, L = int(w.ctx_lens[s]), int(w.ctx_lens[s] + w.q_lens[s])
+        new_k, new_v, tok = [], [], np.arange(cu[s], cu[s + 1])
+        for pos in range(ids.size * w.block_size):
+            bi, sl = pos // w.block_size, pos % w.block_size
+            if c <= pos < L:
+                new_k.append(dev[bi, 0, :, sl])
+                new_v.append(dev[bi, 1, :, sl])
+            else:  # prior context and slots past the end: untouched, bit for bit
+                assert np.array_equal(dev[bi, :, :, sl], ref_blocks[bi, :, :, sl]), f"slot {pos} of seq {s}"
+        near(np.stack(new_k), k_ref[tok], pair_mag(k[tok]), f"new K of seq {s}")
+        near(np.stack(new_v), v[tok], 0.0, f"new V of seq {s}")
     assert_close(bf16_to_f64(to_bits(out)), ref, w.name)
     _free(cache, batch)

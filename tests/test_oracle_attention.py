@@ -225,3 +225,30 @@ def test_pass_without_rotary_appends_the_bits_and_attends_with_q_itself():
                 e = np.exp(z - z.max())
                 ref = (e[:, None] * Vf[:p + 1, hk]).sum(0) / e.sum()
                 assert np.allclose(out[cu[s] + j, h], ref, rtol=0, atol=1e-12)
+
+
+def test_qkv_projection_against_term_by_term_sums():
+    """The projection oracle on a tiny case against sums written out term by
+    term (math.fsum, exact) and a brute-force nearest-bf16 rounding."""
+    import math
+    from oracle import qkv_projection
+    from oracle.bf16 import bf16_bits_to_f64 as widen
+    rng = np.random.default_rng(5)
+    T, hidden, hq, hkv, d = 3, 64, 2, 1, 4
+    x = f32_to_bf16_bits(rng.standard_normal((T, hidden)).astype(np.float32))
+    w = f32_to_bf16_bits((rng.standard_normal(((hq + 2 * hkv) * d, hidden)) / 8).astype(np.float32))
+    q, k, v = qkv_projection(x, w, hq, hkv, d)
+    assert q.shape == (T, hq, d) and k.shape == (T, hkv, d) and v.shape == (T, hkv, d)
+    allv = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    fin = allv[np.isfinite(widen(allv))]
+    grid = widen(fin)
+    xs, ws = widen(x), widen(w)
+    out = np.concatenate([q.reshape(T, -1), k.reshape(T, -1), v.reshape(T, -1)], axis=1)
+    for t in range(T):
+        for j in range(ws.shape[0]):
+            exact = math.fsum(float(xs[t, i]) * float(ws[j, i]) for i in range(hidden))
+            dist = np.abs(grid - exact)
+            best = fin[dist == dist.min()]
+            # ties go to the even pattern
+            want = best[0] if len(best) == 1 else best[(best & 1) == 0][0]
+            assert out[t, j] == want, (t, j)
