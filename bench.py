@@ -609,6 +609,123 @@ def run_qkv_fused(args, w):
     return 0
 
 
+class BlockAllocator:
+    """Free list over the pool's block ids (host side of the paged cache):
+    a sequence gets blocks as its context grows and returns them when it
+    finishes."""
+
+    def __init__(self, n_blocks, block_size, seed=0):
+        ids = np.random.default_rng(seed).permutation(n_blocks)
+        self.free = [int(b) for b in ids]
+        self.B = block_size
+        self.owned = {}
+
+    def ensure(self, rid, length):
+        have = self.owned.setdefault(rid, [])
+        need = -(-length // self.B)
+        while len(have) < need:
+            if not self.free:
+                raise RuntimeError("block pool exhausted")
+            have.append(self.free.pop())
+        return have
+
+    def release(self, rid):
+        self.free.extend(self.owned.pop(rid, []))
+
+
+def run_serve_sim(args):
+    """A timed Dynamic SplitFuse loop with attention only (no weights): the
+    composer's closed loop of synthetic clients (32 active of 512 requests,
+    prompt ~N(2600, 30 %), output ~N(60, 30 %), budget 2048: the card's
+    workload, Key points) drives put + rotary/append + attention on one GPU
+    at the Llama-2-7B attention shape, with blocks taken from a free list as
+    contexts grow and returned when a request finishes; the cache is built
+    through the API, chunk by chunk. Each iteration's device time (CUDA
+    events) advances a clock; a request arrives when it becomes active, gets
+    its first token at the end of the iteration that completes its prompt
+    and one more at the end of every later iteration. One JSON line (kind
+    "serve_sim"): throughput, percentiles of time to first token and of the
+    mean time per output token, and the requests per second that meet the
+    latency targets (--sla-ttft-ms, --sla-tpot-ms)."""
+    import torch
+    from ragged_paged_kv_b200 import fg, workloads as W
+    dev = torch.device("cuda", 0)
+    Hq = Hkv = 32
+    d, B, budget = 128, 64, 2048
+    n_blocks = 4096
+    cache = fg.KVCache(B, n_blocks, Hkv, d, device=dev)
+    alloc = BlockAllocator(n_blocks, B, seed=1)
+    batch = fg.RaggedBatch(budget, 64, 128)
+    g = torch.Generator(device=dev).manual_seed(3)
+    q = torch.randn((budget, Hq, d), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((budget, Hkv, d), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((budget, Hkv, d), generator=g, device=dev).to(torch.bfloat16)
+    q_rot, out = torch.empty_like(q), torch.empty_like(q)
+    stream = torch.cuda.Stream(device=dev)
+    scale = 1.0 / d ** 0.5
+    events = []
+    arrive = {rid: 0.0 for rid in range(32)}
+    first, last, n_out = {}, {}, {}
+    clock = 0.0
+    iters = tokens = 0
+    seen = 0
+
+    def settle():
+        # the composer reports an iteration's outcome when it is resumed for
+        # the next one: tokens produced (at the clock's current value, the end
+        # of that iteration), requests that left and those that joined
+        nonlocal seen
+        for _, produced, joined, left in events[seen:]:
+            for r, is_first in produced:
+                if is_first:
+                    first[r] = clock
+                last[r] = clock
+                n_out[r] = n_out.get(r, 0) + 1
+            for r in left:
+                alloc.release(r)
+            for r in joined:
+                arrive[r] = clock
+        seen = len(events)
+
+    for it, bt in W.splitfuse_schedule(seed=2, budget=budget, events=events):
+        settle()
+        rids = np.array([b[0] for b in bt], np.int32)
+        ql = np.array([b[1] for b in bt], np.int32)
+        cl = np.array([b[2] for b in bt], np.int32)
+        tabs = [alloc.ensure(int(r), int(c + n)) for r, n, c in zip(rids, ql, cl)]
+        tab = np.full((len(bt), max(len(t) for t in tabs)), -1, np.int32)
+        for i, t in enumerate(tabs):
+            tab[i, :len(t)] = t
+        T = int(ql.sum())
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        batch.put(cache, rids, ql, cl, tab, stream)
+        fg.rotary_kv_append(cache, batch, q[:T], k[:T], v[:T], q_rot[:T], Hq, 10000.0, stream)
+        fg.ragged_attention(cache, batch, q_rot[:T], out[:T], Hq, scale, 0, stream)
+        e1.record(stream)
+        e1.synchronize()
+        clock += e0.elapsed_time(e1)
+        iters += 1
+        tokens += T
+    settle()
+    batch.device_status(stream)
+    done = sorted(first)
+    ttft = np.array([first[r] - arrive[r] for r in done])
+    tpot = np.array([(last[r] - first[r]) / (n_out[r] - 1) for r in done if n_out[r] > 1])
+    meets = [r for r in done if first[r] - arrive[r] <= args.sla_ttft_ms and
+             (n_out[r] <= 1 or (last[r] - first[r]) / (n_out[r] - 1) <= args.sla_tpot_ms)]
+    pct = lambda a, p: float(np.percentile(a, p)) if len(a) else None
+    print(json.dumps({
+        "kind": "serve_sim", "workload": "Llama-2-7B attention shape, 32 active of 512 requests, budget 2048",
+        "iterations": iters, "tokens": tokens, "requests": len(done), "device_s": clock / 1e3,
+        "tokens_per_s": tokens / clock * 1e3, "requests_per_s": len(done) / clock * 1e3,
+        "ttft_ms": {"p50": pct(ttft, 50), "p95": pct(ttft, 95)},
+        "tpot_ms": {"p50": pct(tpot, 50), "p95": pct(tpot, 95)},
+        "sla": {"ttft_ms": args.sla_ttft_ms, "tpot_ms": args.sla_tpot_ms,
+                "effective_requests_per_s": len(meets) / clock * 1e3}}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -623,6 +740,10 @@ def main():
                     help="size the block pool to what the batch uses (small ncu captures)")
     ap.add_argument("--qkv-fused", action="store_true",
                     help="time the fused Q/K/V projection + rotary + append (one GPU; JSON line, no contract line)")
+    ap.add_argument("--serve-sim", action="store_true",
+                    help="timed SplitFuse loop with closed-loop synthetic clients (one GPU; JSON line)")
+    ap.add_argument("--sla-ttft-ms", type=float, default=30.0)
+    ap.add_argument("--sla-tpot-ms", type=float, default=1.0)
     ap.add_argument("--sweep-tokens", action="store_true",
                     help="latency/throughput against tokens per pass (one GPU; JSON lines, no contract line)")
     args = ap.parse_args()
@@ -630,6 +751,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.sweep_tokens:
         return run_token_sweep(args)
+    if args.serve_sim:
+        return run_serve_sim(args)
     from ragged_paged_kv_b200 import workloads as W
     if args.config == 3 and args.impl == "fg":
         import torch

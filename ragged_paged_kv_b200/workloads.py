@@ -238,7 +238,8 @@ class _Req:
 
 
 def splitfuse_schedule(seed: int, budget: int = 2048, n_active: int = 32, n_total: int = 512,
-                       prompt_mean: float = 2600.0, out_mean: float = 60.0, rel_sd: float = 0.3):
+                       prompt_mean: float = 2600.0, out_mean: float = 60.0, rel_sd: float = 0.3,
+                       events: list | None = None):
     """Yield (iteration, [(rid, q_len, ctx_len), ...]) for a closed loop of
     synthetic clients under a fixed token budget.
 
@@ -253,6 +254,10 @@ def splitfuse_schedule(seed: int, budget: int = 2048, n_active: int = 32, n_tota
          iteration and the next arrival takes its place.
     Prompt length P = max(1, round(N(2600, 780))), output length
     G = max(1, round(N(60, 18))).
+    If `events` is a list, each iteration appends (iteration, produced,
+    joined, left) to it after the batch has been consumed: the (rid,
+    is_first_token) pairs of the tokens the iteration produced, the requests
+    that became active for the next iteration and those that finished.
     """
     rng = np.random.default_rng(np.random.SeedSequence(seed, spawn_key=(_KIND_LENS,)))
     P = np.maximum(1, np.rint(rng.normal(prompt_mean, rel_sd * prompt_mean, n_total))).astype(int)
@@ -278,6 +283,7 @@ def splitfuse_schedule(seed: int, budget: int = 2048, n_active: int = 32, n_tota
         yield it, batch
         by_id = {b[0]: b for b in batch}
         still = []
+        produced = []
         for r in active:
             b = by_id.get(r.rid)
             if b is not None:
@@ -285,15 +291,22 @@ def splitfuse_schedule(seed: int, budget: int = 2048, n_active: int = 32, n_tota
                     r.done += b[1]
                     if r.done == r.prompt:
                         r.gen = 1
+                        produced.append((r.rid, True))
                 else:
                     r.gen += 1
+                    produced.append((r.rid, False))
             if r.done == r.prompt and r.gen >= r.out:
                 continue
             still.append(r)
+        left_ids = [r.rid for r in active if r not in still]
         active = still
+        joined = []
         while len(active) < n_active and nxt < n_total:
             active.append(_Req(nxt, int(P[nxt]), int(G[nxt])))
+            joined.append(nxt)
             nxt += 1
+        if events is not None:
+            events.append((it, produced, joined, left_ids))
         it += 1
 
 
