@@ -186,10 +186,13 @@ fg_status fg_kv_append(fg_kv_cache* cache, const fg_ragged_batch* batch, const v
  *   out = sum_k exp(z_k - m) V_k / sum_k exp(z_k - m),
  *   z_k = softmax_scale * <q, K_k>,  m = max_k z_k,
  * with bf16 operands, fp32 accumulation and fp32 softmax. Must follow the
- * fg_rotary_kv_append of the same batch on the same stream (a token sees its
- * own K/V). Long contexts are split across thread blocks and merged by a
- * log-sum-exp combine; the split workspace is owned by the batch handle and
- * grown (cudaMalloc, after a device synchronize) when a pass needs more. */
+ * append of the same batch (fg_rotary_kv_append, fg_kv_append or
+ * fg_qkv_rotary_kv_append) on the same stream (a token sees its own K/V).
+ * Long contexts are split across thread blocks and merged by a log-sum-exp
+ * combine. The split workspace and the work-plan buffer are owned by the
+ * batch handle and grown with stream-ordered allocation (cudaMallocAsync on
+ * `stream`) when a pass needs more; the host builds the plan and uploads it
+ * through pinned staging each time the batch or (n_q_heads, window) changes. */
 fg_status fg_ragged_attention(const fg_kv_cache* cache, fg_ragged_batch* batch, const void* q_rot,
                               void* out, int32_t n_q_heads, float softmax_scale,
                               int32_t sliding_window, void* stream);
@@ -246,13 +249,17 @@ fg_status fg_attention_kernel_ms(fg_ragged_batch* batch, float ms[4]);
  * launches. reset != 0 zeroes the counters after reading them. */
 fg_status fg_host_profile_us(fg_ragged_batch* batch, double out[8], int32_t reset);
 
-/* Scheduling of one attention call that has both one-token decode units and
- * prompt-chunk query tiles. enable == 0 (default): the two kernels run one
- * after the other on the caller's stream, each with the whole GPU (two CTAs
- * per SM). enable != 0: the query-tile kernel runs on a second,
- * high-priority stream beside the decode kernel, each sized for one CTA per
- * SM. On a B200 the default is faster (the hardware may place two CTAs of
- * one kernel on an SM, which unbalances the persistent grids). Results are
+/* Scheduling of one attention call that has both one-token decodes (d = 128,
+ * on the tensor-core decode kernel) and prompt-chunk query tiles.
+ * enable == 0 (default): the query-tile kernel, then the decode kernel (its
+ * CTAs take SMs as the query-tile CTAs leave), then the combine, on the
+ * caller's stream. enable != 0: the two kernels run side by side, the query
+ * tiles on a second, high-priority stream: a cost model picks K, the
+ * query-tile kernel takes the SMs with id < K and the decode kernel the
+ * rest, and decode CTAs move onto the first K SMs once every query tile has
+ * been claimed; when the model predicts no gain the call runs as with
+ * enable == 0. On a B200 the default is faster on the measured batches (the
+ * decode kernel needs nearly every SM to reach HBM speed). Results are
  * identical either way. */
 fg_status fg_ragged_batch_set_overlap(fg_ragged_batch* batch, int32_t enable);
 

@@ -18,10 +18,14 @@
 // stage raises it by more than 2^8; per-thread partial sums are reduced once
 // per unit.
 //
-// The kernel is persistent (units b, b + grid, ... of a longest-first list)
-// and streams K and V through one ring of 32 KB slots (K and V of a stage
-// take consecutive slots). At about 109 KB of shared memory and 64 TMEM
-// columns it fits beside a prefill CTA of attn_tc_kernel on the same SM.
+// The kernel is persistent, two CTAs per SM (about 109 KB of shared memory
+// and 64 TMEM columns each): the TMA warp takes units from a global counter
+// over a longest-first list and hands them to the other roles through a
+// small queue, and K and V stream through one ring of 32 KB slots (K and V
+// of a stage take consecutive slots). Launched behind the query-tile kernel
+// with programmatic dependent launch, its CTAs take SMs as that kernel's
+// CTAs leave; it does not read that kernel's results, but waits for it
+// before its own CTAs end so that the combine launched behind it sees both.
 // Every wait is bounded.
 #include <cuda.h>
 
