@@ -112,8 +112,14 @@ fg_status fg_ragged_batch_create(int32_t max_tokens, int32_t max_seqs, int32_t m
  * written twice, no block repeated within one table, no new token written
  * into a slot that another sequence of the batch reads, distinct seq_ids
  * (FG_ERR_ALIAS). The packed metadata is copied to the device
- * asynchronously on `stream` from a pinned staging buffer; a later put on
- * the same handle first waits for that copy. */
+ * asynchronously from a pinned staging buffer, into one half of a double
+ * buffer, on a copy stream of the handle's own; `stream` waits for that copy,
+ * so work queued on it after the put sees the new pass. The copy itself waits
+ * only for the work queued on `stream` before the previous put (the last
+ * work that read the same half), so it runs while the device still works on
+ * the previous pass. Keep every call that uses a pass on the stream of its
+ * put, or order other streams after it. A put on the same handle may wait on
+ * the host for the copy of the put two before it. */
 fg_status fg_ragged_batch_put(fg_ragged_batch* batch, const fg_kv_cache* cache, int32_t n_seqs,
                               const int32_t* seq_ids, const int32_t* q_lens,
                               const int32_t* ctx_lens, const int32_t* block_tables,
@@ -192,7 +198,10 @@ fg_status fg_kv_append(fg_kv_cache* cache, const fg_ragged_batch* batch, const v
  * combine. The split workspace and the work-plan buffer are owned by the
  * batch handle and grown with stream-ordered allocation (cudaMallocAsync on
  * `stream`) when a pass needs more; the host builds the plan and uploads it
- * through pinned staging each time the batch or (n_q_heads, window) changes. */
+ * through pinned staging each time the batch or (n_q_heads, window) changes,
+ * into one half of a double buffer on the handle's copy stream, the way
+ * fg_ragged_batch_put uploads the metadata (`stream` waits for the copy, the
+ * copy for the work queued on `stream` before the previous upload). */
 fg_status fg_ragged_attention(const fg_kv_cache* cache, fg_ragged_batch* batch, const void* q_rot,
                               void* out, int32_t n_q_heads, float softmax_scale,
                               int32_t sliding_window, void* stream);

@@ -110,6 +110,74 @@ struct Staging {
   }
 };
 
+// A device buffer with two halves used in turn by successive uploads, so
+// that the upload of the next pass's data (on the handle's copy stream) runs
+// while the device still works on the current pass. rel[i] marks, on the
+// caller's stream, the end of the work queued while half i was current;
+// ready[i] the end of the copy into it, which the caller's stream waits for.
+struct DevDouble {
+  void* buf[2] = {nullptr, nullptr};
+  size_t cap[2] = {0, 0};
+  cudaEvent_t rel[2] = {nullptr, nullptr};
+  cudaEvent_t ready[2] = {nullptr, nullptr};
+  bool rel_set[2] = {false, false};
+  int cur = -1;
+
+  // Makes the other half current-to-be: sized for `need` bytes (grown on
+  // `strm` with stream-ordered allocation, or with cudaMalloc when `sync`),
+  // and `copy` ordered after the last use of it. Returns its index.
+  fg_status begin(size_t need, bool sync, cudaStream_t strm, cudaStream_t copy, int* out) {
+    for (int i = 0; i < 2; ++i) {
+      if (!rel[i]) FG_CUDA(cudaEventCreateWithFlags(&rel[i], cudaEventDisableTiming));
+      if (!ready[i]) FG_CUDA(cudaEventCreateWithFlags(&ready[i], cudaEventDisableTiming));
+    }
+    if (cur >= 0) {
+      FG_CUDA(cudaEventRecord(rel[cur], strm));
+      rel_set[cur] = true;
+    }
+    const int i = cur < 0 ? 0 : cur ^ 1;
+    if (need > cap[i]) {
+      const size_t c = sync ? need : std::max<size_t>(need + need / 2, 1 << 16);
+      if (sync) {
+        if (buf[i]) FG_CUDA(cudaFree(buf[i]));
+        buf[i] = nullptr;
+        FG_CUDA(cudaMalloc(&buf[i], c));
+      } else {
+        if (buf[i]) FG_CUDA(cudaFreeAsync(buf[i], strm));
+        buf[i] = nullptr;
+        FG_CUDA(cudaMallocAsync(&buf[i], c, strm));
+        FG_CUDA(cudaEventRecord(rel[i], strm));
+        rel_set[i] = true;
+      }
+      cap[i] = c;
+    }
+    if (rel_set[i]) FG_CUDA(cudaStreamWaitEvent(copy, rel[i], 0));
+    *out = i;
+    return FG_OK;
+  }
+  // The copy into half i is queued on `copy`: make it current and order
+  // `strm` after the copy.
+  fg_status commit(int i, cudaStream_t strm, cudaStream_t copy) {
+    FG_CUDA(cudaEventRecord(ready[i], copy));
+    FG_CUDA(cudaStreamWaitEvent(strm, ready[i], 0));
+    cur = i;
+    return FG_OK;
+  }
+  void* current() const { return cur < 0 ? nullptr : buf[cur]; }
+  // Call with the device idle.
+  void release() {
+    for (int i = 0; i < 2; ++i) {
+      if (buf[i]) cudaFree(buf[i]);
+      if (rel[i]) cudaEventDestroy(rel[i]);
+      if (ready[i]) cudaEventDestroy(ready[i]);
+      buf[i] = nullptr;
+      rel[i] = ready[i] = nullptr;
+      cap[i] = 0;
+    }
+    cur = -1;
+  }
+};
+
 }  // namespace
 
 struct fg_kv_cache {
@@ -133,10 +201,12 @@ struct fg_kv_cache {
 struct fg_ragged_batch {
   int32_t max_tokens = 0, max_seqs = 0, max_blocks_per_seq = 0;
   int device = -1;
-  // device metadata + error word
-  int32_t* dmeta = nullptr;
+  // device metadata (two halves, see DevDouble) + error word; the uploads of
+  // metadata and plan run on `copy`
+  DevDouble meta;
   size_t dmeta_words = 0;
   int32_t* derr = nullptr;
+  cudaStream_t copy = nullptr;
   // The persistent kernels' next-unit counters sit in the 256 bytes after
   // the plan in the plan buffer; an upload of a new plan zeroes them too
   // (ctr_fresh), otherwise a memset does before the kernels run.
@@ -154,8 +224,7 @@ struct fg_ragged_batch {
   // attention plan
   fg::Plan plan;
   uint64_t plan_key[4] = {~0ull, 0, 0, 0};
-  void* dplan = nullptr;
-  size_t dplan_bytes = 0;
+  DevDouble dplan;
   Staging plan_stage;
   int32_t last_launches = 0;
   // second stream: tensor-core tiles run beside the decode kernel
@@ -341,13 +410,14 @@ extern "C" fg_status fg_ragged_batch_create(int32_t max_tokens, int32_t max_seqs
 
 extern "C" fg_status fg_ragged_batch_destroy(fg_ragged_batch* b) {
   if (!b) return FG_OK;
-  if (b->dmeta || b->dplan || b->ws) cudaDeviceSynchronize();
+  if (b->derr || b->dplan.cur >= 0 || b->ws) cudaDeviceSynchronize();
   b->meta_stage.release();
   b->plan_stage.release();
-  if (b->dmeta) cudaFree(b->dmeta);
+  b->meta.release();
+  b->dplan.release();
   if (b->derr) cudaFree(b->derr);
-  if (b->dplan) cudaFree(b->dplan);
   if (b->ws) cudaFree(b->ws);
+  if (b->copy) cudaStreamDestroy(b->copy);
   for (cudaEvent_t e : b->tev)
     if (e) cudaEventDestroy(e);
   if (b->aux) cudaStreamDestroy(b->aux);
@@ -466,16 +536,25 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
     return st;
   }
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
-  if (!b->dmeta) {
+  if (!b->derr) {
     b->dmeta_words = 3 * (size_t)b->max_seqs + 2 + (size_t)b->max_tokens +
                      (size_t)b->max_seqs * b->max_blocks_per_seq;
     FG_CUDA(cudaGetDevice(&b->device));
-    FG_CUDA(cudaMalloc(&b->dmeta, b->dmeta_words * 4));
-    FG_CUDA(cudaMalloc(&b->derr, 4));
-    FG_CUDA(cudaMemset(b->derr, 0, 4));
+    if (!b->copy) {
+      int lo = 0, hi = 0;
+      FG_CUDA(cudaDeviceGetStreamPriorityRange(&lo, &hi));
+      FG_CUDA(cudaStreamCreateWithPriority(&b->copy, cudaStreamNonBlocking, hi));
+    }
     st = b->meta_stage.reserve(b->dmeta_words * 4);
     if (st) return st;
+    FG_CUDA(cudaMalloc(&b->derr, 4));
+    FG_CUDA(cudaMemset(b->derr, 0, 4));
   }
+  // the half of the device buffer this pass uses; its copy waits for the
+  // work queued on `stream` before the previous put (the last pass that read it)
+  int half = 0;
+  st = b->meta.begin(b->dmeta_words * 4, true, strm, b->copy, &half);
+  if (st) return st;
   // pack: cu_q[S+1] ctx[S] bt_off[S+1] tok_seq[T] bt[nblk]
   const size_t words = 3 * (size_t)S + 2 + (size_t)T + (size_t)nblk;
   void* hp = nullptr;
@@ -501,10 +580,12 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
     std::memcpy(bb + bo[s], bt + (int64_t)s * stride, (size_t)nb * 4);
     for (int32_t j = 0; j < ql[s]; ++j) ts[cu[s] + j] = s;
   }
-  st = b->meta_stage.copy(slot, b->dmeta, words * 4, strm);
+  int32_t* d = static_cast<int32_t*>(b->meta.buf[half]);
+  st = b->meta_stage.copy(slot, d, words * 4, b->copy);
+  if (st) return st;
+  st = b->meta.commit(half, strm, b->copy);
   if (st) return st;
   b->hprof[0] += now_us() - t_in;
-  int32_t* d = b->dmeta;
   b->view.cu_q = d;
   b->view.ctx = d + S + 1;
   b->view.bt_off = d + 2 * S + 1;
@@ -701,20 +782,17 @@ fg_status prepare_plan(fg_ragged_batch* b, const fg_kv_cache* c, int32_t g, int3
                        bool use_tc, cudaStream_t strm) {
   const uint64_t key[4] = {b->put_gen, (uint64_t)g, (uint64_t)(uint32_t)window,
                            (uint64_t)c->head_dim | ((uint64_t)use_tc << 32)};
-  if (std::equal(key, key + 4, b->plan_key) && b->dplan) return FG_OK;
+  if (std::equal(key, key + 4, b->plan_key) && b->dplan.current()) return FG_OK;
   const double t_p = now_us();
   fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc,
                  sm_count(), &b->plan);
   b->hprof[4] += now_us() - t_p;
   const size_t bytes = b->plan.bytes() + 256;  // plan, then the unit counters
-  if (bytes > b->dplan_bytes) {
-    if (b->dplan) FG_CUDA(cudaFreeAsync(b->dplan, strm));
-    b->dplan = nullptr;
-    const size_t cap = std::max<size_t>(bytes + bytes / 2, 1 << 16);
-    FG_CUDA(cudaMallocAsync(&b->dplan, cap, strm));
-    b->dplan_bytes = cap;
-  }
-  fg_status st = b->plan_stage.reserve(b->dplan_bytes);
+  // the other half of the plan buffer, once the last pass that used it is done
+  int half = 0;
+  fg_status st = b->dplan.begin(bytes, false, strm, b->copy, &half);
+  if (st) return st;
+  st = b->plan_stage.reserve(b->dplan.cap[half]);
   if (st) return st;
   void* hp = nullptr;
   int slot = 0;
@@ -724,7 +802,9 @@ fg_status prepare_plan(fg_ragged_batch* b, const fg_kv_cache* c, int32_t g, int3
   if (st) return st;
   b->plan.pack(hp);
   std::memset(static_cast<char*>(hp) + b->plan.bytes(), 0, 256);
-  st = b->plan_stage.copy(slot, b->dplan, bytes, strm);
+  st = b->plan_stage.copy(slot, b->dplan.buf[half], bytes, b->copy);
+  if (st) return st;
+  st = b->dplan.commit(half, strm, b->copy);
   if (st) return st;
   b->ctr_fresh = true;
   std::copy(key, key + 4, b->plan_key);
@@ -799,7 +879,7 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   b->last_launches = (P.n_general > 0) + (P.n_decode > 0) + (P.n_tc > 0) + (P.n_dtc > 0) +
                      (P.n_combine > 0);
-  const char* base = static_cast<const char*>(b->dplan);
+  const char* base = static_cast<const char*>(b->dplan.current());
   const CacheView cv = cache_view(c);
   const auto* qr = static_cast<const __nv_bfloat16*>(q_rot);
   auto* o = static_cast<__nv_bfloat16*>(out);
@@ -830,7 +910,7 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
     tc_stream = b->aux;
   }
   // the persistent kernels' unit counters start at zero
-  int* ctr = reinterpret_cast<int*>(static_cast<char*>(b->dplan) + P.bytes());
+  int* ctr = reinterpret_cast<int*>(static_cast<char*>(b->dplan.current()) + P.bytes());
   if ((P.n_tc || P.n_dtc) && !b->ctr_fresh) FG_CUDA(cudaMemsetAsync(ctr, 0, 8, strm));
   b->ctr_fresh = false;
   // programmatic dependent launch along the chain query tiles -> decode ->
