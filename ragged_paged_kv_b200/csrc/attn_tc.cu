@@ -530,6 +530,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         const int row = x.row0 + rr / g;
         const int qh = x.h * g + (rr % g);
         const float inv = l > 0.f ? 1.f / l : 0.f;
+        const bool wide = ((reinterpret_cast<uintptr_t>(a.out) | reinterpret_cast<uintptr_t>(a.part_o)) & 31u) == 0;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t o[D / 2];
@@ -539,25 +540,41 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
                            *reinterpret_cast<uint32_t(*)[32]>(&o[c * 32]));
           ptx::tmem_ld_wait();
           if (!row_ok) continue;
+          // a thread writes its own row, so each store instruction touches
+          // 32 rows; 32-byte stores (when the bases allow) halve their number
           if (x.part < 0) {
-            uint4* dst = reinterpret_cast<uint4*>(a.out + ((int64_t)row * a.Hq + qh) * D + hh * (D / 2));
+            __nv_bfloat16* dst = a.out + ((int64_t)row * a.Hq + qh) * D + hh * (D / 2);
 #pragma unroll
-            for (int q4 = 0; q4 < D / 16; ++q4) {
-              uint32_t w[4];
+            for (int q8 = 0; q8 < D / 32; ++q8) {
+              uint32_t w[8];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(o[q4 * 8 + 2 * e]) * inv,
-                                                          __uint_as_float(o[q4 * 8 + 2 * e + 1]) * inv);
+              for (int e = 0; e < 8; ++e) {
+                __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(o[q8 * 16 + 2 * e]) * inv,
+                                                          __uint_as_float(o[q8 * 16 + 2 * e + 1]) * inv);
                 w[e] = *reinterpret_cast<uint32_t*>(&pr);
               }
-              dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+              if (wide) {
+                ptx::st_global_v8(dst + q8 * 16, w);
+              } else {
+                uint4* d4 = reinterpret_cast<uint4*>(dst + q8 * 16);
+                d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              }
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(a.part_o + (int64_t)(x.part + rr) * D + hh * (D / 2));
+            float* dst = a.part_o + (int64_t)(x.part + rr) * D + hh * (D / 2);
 #pragma unroll
-            for (int q4 = 0; q4 < D / 8; ++q4)
-              dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
-                                    __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
+            for (int q8 = 0; q8 < D / 16; ++q8) {
+              if (wide) {
+                ptx::st_global_v8(dst + q8 * 8, &o[q8 * 8]);
+              } else {
+                float4* d4 = reinterpret_cast<float4*>(dst + q8 * 8);
+                d4[0] = make_float4(__uint_as_float(o[8 * q8]), __uint_as_float(o[8 * q8 + 1]),
+                                    __uint_as_float(o[8 * q8 + 2]), __uint_as_float(o[8 * q8 + 3]));
+                d4[1] = make_float4(__uint_as_float(o[8 * q8 + 4]), __uint_as_float(o[8 * q8 + 5]),
+                                    __uint_as_float(o[8 * q8 + 6]), __uint_as_float(o[8 * q8 + 7]));
+              }
+            }
           }
         }
         if (row_ok && x.part >= 0) {
