@@ -567,10 +567,11 @@ def run_token_sweep(args):
 
 
 def run_qkv_fused(args, w):
-    """The Q/K/V projection fused with rotary + append on the headline batch's
-    tokens at Llama-2-7B width (hidden 4096, 96 heads of 128 out): one JSON
-    line with its device time, TFLOP/s and fraction of the measured bf16
-    peak (kind "qkv_fused", not the contract line)."""
+    """The Q/K/V projection fused with rotary + append, and the output
+    projection, on the headline batch's tokens at Llama-2-7B width (hidden
+    4096; 96 heads of 128 out, then 4096 -> 4096): one JSON line per GEMM with
+    its device time, TFLOP/s and fraction of the measured bf16 peak (kinds
+    "qkv_fused" and "out_proj", not the contract line)."""
     import torch
     from ragged_paged_kv_b200 import fg, fixtures
     dev = torch.device("cuda", 0)
@@ -604,6 +605,29 @@ def run_qkv_fused(args, w):
     flops = 2.0 * w.n_tokens * hidden * n_out
     hbm, tf, src = load_peaks()
     print(json.dumps({"kind": "qkv_fused", "workload": f"{w.name}: T={w.n_tokens}, hidden={hidden}, out={n_out}",
+                      "ms": ms, "tflops": flops / ms / 1e9, "peak_tflops": tf, "frac": flops / ms / 1e9 / tf,
+                      "peak_source": src}), flush=True)
+
+    # the output projection: the attention output [T, Hq d] times W_o^T
+    k_in = w.n_q_heads * w.head_dim
+    o = torch.randn((w.n_tokens, k_in), generator=g, device=dev).to(torch.bfloat16)
+    wo = (torch.randn((hidden, k_in), generator=g, device=dev) / k_in ** 0.5).to(torch.bfloat16)
+    y = torch.empty((w.n_tokens, hidden), dtype=torch.bfloat16, device=dev)
+    evs = []
+    for i in range(args.warmup + args.steps):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            flush.sum()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        fg.output_projection(batch, o, wo, y, stream)
+        e[1].record(stream)
+        if i >= args.warmup:
+            evs.append(e)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    flops = 2.0 * w.n_tokens * k_in * hidden
+    print(json.dumps({"kind": "out_proj", "workload": f"{w.name}: T={w.n_tokens}, in={k_in}, out={hidden}",
                       "ms": ms, "tflops": flops / ms / 1e9, "peak_tflops": tf, "frac": flops / ms / 1e9 / tf,
                       "peak_source": src}), flush=True)
     return 0
@@ -739,7 +763,7 @@ def main():
     ap.add_argument("--compact-pool", action="store_true",
                     help="size the block pool to what the batch uses (small ncu captures)")
     ap.add_argument("--qkv-fused", action="store_true",
-                    help="time the fused Q/K/V projection + rotary + append (one GPU; JSON line, no contract line)")
+                    help="time the fused Q/K/V projection + rotary + append and the output projection (one GPU; JSON lines, no contract line)")
     ap.add_argument("--serve-sim", action="store_true",
                     help="timed SplitFuse loop with closed-loop synthetic clients (one GPU; JSON line)")
     ap.add_argument("--sla-ttft-ms", type=float, default=30.0)

@@ -233,6 +233,25 @@ fg_status fg_ragged_attention_noalloc(const fg_kv_cache* cache, fg_ragged_batch*
                                       const void* q_rot, void* out, int32_t n_q_heads,
                                       float softmax_scale, int32_t sliding_window, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* After step 3: the layer's output projection                               */
+/* ------------------------------------------------------------------------ */
+
+/* y = attn_out w_o^T for the batch's T tokens: attn_out device
+ * [T][in_features] bf16 (the attention output [T][n_q_heads][d] viewed as
+ * rows of n_q_heads * d), w_o device [out_features][in_features] bf16 (the
+ * layout of a linear layer's weight), y device [T][out_features] bf16. Each
+ * output is the fp32-accumulated sum rounded once to bf16 (ties to even), as
+ * a linear layer with bf16 output returns it; fp32 sums in another order can
+ * round a value to the neighbouring bf16 of the exact sum's rounding. The
+ * pages run whole transformer layers (Key points); this is the GEMM that
+ * follows the attention in each of them. in_features and out_features must
+ * be positive multiples of 64 (FG_ERR_UNSUPPORTED); the pointers 16-byte
+ * aligned (FG_ERR_INVALID_ARG). The batch must hold a valid put (its T is
+ * used; nothing else). Asynchronous on `stream`; allocates nothing. */
+fg_status fg_output_projection(const fg_ragged_batch* batch, const void* attn_out, const void* w_o,
+                               int32_t in_features, int32_t out_features, void* y, void* stream);
+
 /* Work plan of the batch's last fg_ragged_attention call, for profiling:
  * info[0] = general-path units, info[1] = split-KV decode units,
  * info[2] = tensor-core units, info[3] = combine groups, info[4] = partial

@@ -27,7 +27,7 @@ from .bf16 import bf16_bits_to_f64, f64_to_bf16_bits
 from .rotary import inv_freq, rope_table, rotate_half
 from .paged_cache import PagedCache, append_kv, token_positions
 from .attention import attend_contiguous, ragged_attention
-from .projection import qkv_projection
+from .projection import linear, qkv_projection
 
 __all__ = [
     "bf16_bits_to_f64", "f64_to_bf16_bits", "inv_freq", "rope_table", "rotate_half",

@@ -1162,5 +1162,31 @@ extern "C" fg_status fg_qkv_rotary_kv_append(fg_kv_cache* c, const fg_ragged_bat
   return FG_OK;
 }
 
+extern "C" fg_status fg_output_projection(const fg_ragged_batch* b, const void* attn_out, const void* w_o,
+                                          int32_t in_features, int32_t out_features, void* y, void* stream) {
+  if (!b) return fail(FG_ERR_INVALID_ARG, "batch is NULL");
+  if (!b->cache) return fail(FG_ERR_INVALID_ARG, "batch has no valid put");
+  if (in_features < 64 || in_features % 64)
+    return fail(FG_ERR_UNSUPPORTED, "in_features %d is not a positive multiple of 64", in_features);
+  if (out_features < 64 || out_features % 64)
+    return fail(FG_ERR_UNSUPPORTED, "out_features %d is not a positive multiple of 64", out_features);
+  int dev = -1;
+  if (cudaGetDevice(&dev) == cudaSuccess && b->device >= 0 && dev != b->device)
+    return fail(FG_ERR_INVALID_ARG, "current device %d is not the batch's device %d", dev, b->device);
+  if (b->n_tokens == 0) return FG_OK;
+  if (!attn_out || !w_o || !y) return fail(FG_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(attn_out) || !aligned16(w_o) || !aligned16(y))
+    return fail(FG_ERR_INVALID_ARG, "attn_out, w_o and y must be 16-byte aligned");
+  const uint32_t n_tile = out_features % 128 == 0 ? 128 : 64;
+  CUtensorMap tm_x, tm_w;
+  if (!make_rows_map(&tm_x, attn_out, (uint64_t)in_features, (uint64_t)b->n_tokens, 128) ||
+      !make_rows_map(&tm_w, w_o, (uint64_t)in_features, (uint64_t)out_features, n_tile))
+    return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for attn_out or w_o");
+  cudaError_t e = fg::launch_linear_bf16(&tm_x, &tm_w, b->view, static_cast<__nv_bfloat16*>(y), in_features,
+                                         out_features, (int)n_tile, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "output projection launch");
+  return FG_OK;
+}
+
 // Sets the thread-local error text (for entry points defined in other files).
 fg_status fg_set_error(fg_status st, const char* msg) { return fail(st, "%s", msg); }

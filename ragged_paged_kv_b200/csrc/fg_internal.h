@@ -104,6 +104,13 @@ cudaError_t launch_qkv_rotary_append(const void* tm_x, const void* tm_w, const C
                                      const BatchView& batch, __nv_bfloat16* q_rot, const double2* rope,
                                      int n_q_heads, int hidden, cudaStream_t stream);
 
+// y[T][n_out] = x[T][k_len] w[n_out][k_len]^T in bf16 with fp32 accumulation
+// (the layer's output projection); T = batch.n_tokens, n_tile (64 or 128)
+// output features per CTA, tm_x / tm_w 2-D maps with 64 x 128 and
+// 64 x n_tile boxes.
+cudaError_t launch_linear_bf16(const void* tm_x, const void* tm_w, const BatchView& batch, __nv_bfloat16* y,
+                               int k_len, int n_out, int n_tile, cudaStream_t stream);
+
 cudaError_t launch_combine(const BatchView& batch, const CombineItem* items, int n_items,
                            int max_rows, const float* part_o, const float* part_ml,
                            __nv_bfloat16* out, int n_q_heads, int g, int head_dim, bool pdl,

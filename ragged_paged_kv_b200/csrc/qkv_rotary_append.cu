@@ -11,6 +11,11 @@
 // of x and W with 2-D TMA boxes (128-byte swizzle) into a 3-stage ring, warp
 // 1 (one thread) issues the MMAs, warps 2-5 (TMEM lanes 32 (w % 4) ..) run
 // the epilogue. Every wait is bounded.
+//
+// The same kernel with LINEAR = true is the layer's output projection
+// y = o W_o^T (o the attention output viewed as [T, Hq d]): a CTA computes
+// 128 tokens x D output features, and the epilogue rounds them to bf16 and
+// stores them into y.
 #include <cuda.h>
 
 #include <cfloat>
@@ -44,7 +49,9 @@ struct QkvArgs {
   __nv_bfloat16* q_rot;
   const double2* rope;  // the rotary table, see below
   int Hq;
-  int hidden;
+  int hidden;           // the contraction length
+  __nv_bfloat16* y;     // LINEAR: output [T][n_out]
+  int n_out;
 };
 
 // float64 -> bf16 with one rounding (truncate to float, force the last bit on
@@ -64,7 +71,7 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int
   return ok;
 }
 
-template <int D>
+template <int D, bool LINEAR>
 __global__ void __launch_bounds__(192, 2) qkv_rotary_append_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                                   const __grid_constant__ CUtensorMap tm_w,
                                                                   QkvArgs a) {
@@ -149,7 +156,29 @@ __global__ void __launch_bounds__(192, 2) qkv_rotary_append_kernel(const __grid_
       for (int c = 0; c < D / 32; ++c)
         ptx::tmem_ld32(tmem + lane_base + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&acc[c * 32]));
       ptx::tmem_ld_wait();
-      if (t < a.batch.n_tokens) {
+      if (LINEAR && t < a.batch.n_tokens) {
+        // round to bf16, pack pairs, and store the row's D features (32-byte
+        // stores when y and its row pitch allow)
+        __nv_bfloat16* dst = a.y + (int64_t)t * a.n_out + head * D;
+        const bool wide = ((reinterpret_cast<uintptr_t>(a.y) | ((uintptr_t)a.n_out * 2)) & 31u) == 0;
+#pragma unroll
+        for (int q8 = 0; q8 < D / 16; ++q8) {
+          uint32_t w[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(acc[q8 * 16 + 2 * e]),
+                                                      __uint_as_float(acc[q8 * 16 + 2 * e + 1]));
+            w[e] = *reinterpret_cast<uint32_t*>(&pr);
+          }
+          if (wide) {
+            ptx::st_global_v8(dst + q8 * 16, w);
+          } else {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + q8 * 16);
+            d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          }
+        }
+      } else if (!LINEAR && t < a.batch.n_tokens) {
         // the projection's bf16 output, in place (bits in the low half)
 #pragma unroll
         for (int e = 0; e < D; ++e) acc[e] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(acc[e])));
@@ -203,19 +232,19 @@ __global__ void __launch_bounds__(192, 2) qkv_rotary_append_kernel(const __grid_
   }
 }
 
-template <int D>
+template <int D, bool LINEAR>
 cudaError_t launch_qkv_d(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const QkvArgs& args,
                          int n_heads_total, cudaStream_t stream) {
   using C = QkvCfg<D>;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(qkv_rotary_append_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(qkv_rotary_append_kernel<D, LINEAR>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   dim3 grid((args.batch.n_tokens + C::BM - 1) / C::BM, n_heads_total);
-  qkv_rotary_append_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tm_x, tm_w, args);
+  qkv_rotary_append_kernel<D, LINEAR><<<grid, C::kThreads, C::kSmem, stream>>>(tm_x, tm_w, args);
   return cudaGetLastError();
 }
 
@@ -225,12 +254,26 @@ cudaError_t launch_qkv_rotary_append(const void* tm_x, const void* tm_w, const C
                                      const BatchView& batch, __nv_bfloat16* q_rot, const double2* rope,
                                      int n_q_heads, int hidden, cudaStream_t stream) {
   if (batch.n_tokens == 0) return cudaSuccess;
-  QkvArgs args{cache, batch, q_rot, rope, n_q_heads, hidden};
+  QkvArgs args{cache, batch, q_rot, rope, n_q_heads, hidden, nullptr, 0};
   const int heads = n_q_heads + 2 * cache.n_kv_heads;
   const CUtensorMap& x = *static_cast<const CUtensorMap*>(tm_x);
   const CUtensorMap& w = *static_cast<const CUtensorMap*>(tm_w);
-  if (cache.head_dim == 128) return launch_qkv_d<128>(x, w, args, heads, stream);
-  return launch_qkv_d<64>(x, w, args, heads, stream);
+  if (cache.head_dim == 128) return launch_qkv_d<128, false>(x, w, args, heads, stream);
+  return launch_qkv_d<64, false>(x, w, args, heads, stream);
+}
+
+cudaError_t launch_linear_bf16(const void* tm_x, const void* tm_w, const BatchView& batch, __nv_bfloat16* y,
+                               int k_len, int n_out, int n_tile, cudaStream_t stream) {
+  if (batch.n_tokens == 0) return cudaSuccess;
+  QkvArgs args{};
+  args.batch = batch;
+  args.hidden = k_len;
+  args.y = y;
+  args.n_out = n_out;
+  const CUtensorMap& x = *static_cast<const CUtensorMap*>(tm_x);
+  const CUtensorMap& w = *static_cast<const CUtensorMap*>(tm_w);
+  if (n_tile == 128) return launch_qkv_d<128, true>(x, w, args, n_out / 128, stream);
+  return launch_qkv_d<64, true>(x, w, args, n_out / 64, stream);
 }
 
 }  // namespace fg

@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
         "fg_rotary_kv_append": [V, V, V, V, V, V, I32, D, V],
         "fg_kv_append": [V, V, V, V, V],
         "fg_qkv_rotary_kv_append": [V, V, V, V, I32, V, I32, D, V],
+        "fg_output_projection": [V, V, V, I32, I32, V, V],
         "fg_ragged_attention": [V, V, V, V, I32, F, I32, V],
         "fg_ragged_attention_noalloc": [V, V, V, V, I32, F, I32, V],
         "fg_device_status": [V, V],
@@ -260,6 +261,18 @@ def qkv_rotary_kv_append(cache: KVCache, batch: RaggedBatch, x, w_qkv, q_rot, n_
                                          int(x.shape[1]), _dev_ptr(q_rot, "q_rot"), int(n_q_heads),
                                          float(rope_theta), _stream_ptr(stream)),
            "fg_qkv_rotary_kv_append")
+
+
+def output_projection(batch: RaggedBatch, attn_out, w_o, y, stream=None):
+    """The layer's output projection y = attn_out w_o^T (see
+    fg_output_projection): attn_out [T, in] (or [T, Hq, d]), w_o [out, in],
+    y [T, out], all bf16 on the device."""
+    x = attn_out.reshape(attn_out.shape[0], -1) if attn_out.dim() == 3 else attn_out
+    if x.dim() != 2 or w_o.dim() != 2 or x.shape[1] != w_o.shape[1] or tuple(y.shape) != (x.shape[0], w_o.shape[0]):
+        raise ValueError("attn_out must be [T, in], w_o [out, in] and y [T, out]")
+    _check(lib().fg_output_projection(batch.handle, _dev_ptr(x, "attn_out"), _dev_ptr(w_o, "w_o"),
+                                      int(w_o.shape[1]), int(w_o.shape[0]), _dev_ptr(y, "y"),
+                                      _stream_ptr(stream)), "fg_output_projection")
 
 
 def kv_append(cache: KVCache, batch: RaggedBatch, k, v, stream=None):

@@ -372,3 +372,42 @@ def test_fused_qkv_projection_rotary_append(which):
         near(np.stack(new_v), v[tok], 0.0, f"new V of seq {s}")
     assert_close(bf16_to_f64(to_bits(out)), ref, w.name)
     _free(cache, batch)
+
+
+@pytest.mark.parametrize("which", ["tiny_n64", "ragged_n128", "llama7b_width"])
+def test_output_projection(which):
+    """fg_output_projection: y = o W_o^T against the oracle's exactly summed
+    linear layer rounded once to bf16. The GPU's fp32 sums may round a value
+    to the neighbouring bf16, so every word is within the rounding of both
+    sides plus the fp32 accumulation bound, and almost all are identical.
+    The cases cover 64- and 128-wide output tiles and a token count with a
+    ragged last 128-row tile."""
+    from oracle import linear
+    # (tokens as q_lens of a few sequences, in_features, out_features)
+    shapes = {"tiny_n64": ([40, 1, 1, 22], 256, 192),
+              "ragged_n128": ([300, 1, 17], 512, 256),
+              "llama7b_width": ([517, 1, 1, 11], 4096, 4096)}
+    q_lens, k_in, n_out = shapes[which]
+    S = len(q_lens)
+    w = W._make("proj_" + which, 4, 4, 64, 16, list(range(S)), q_lens, [0] * S, seed=31,
+                budget=int(sum(q_lens)))
+    rng = np.random.default_rng(32)
+    x_bits = W.f32_to_bf16_bits(rng.standard_normal((w.n_tokens, k_in)).astype(np.float32))
+    w_bits = W.f32_to_bf16_bits((rng.standard_normal((n_out, k_in)) / np.sqrt(k_in)).astype(np.float32))
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+    batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+    batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables)
+    xd = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    wd = torch.from_numpy(w_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    y = torch.full((w.n_tokens, n_out), float("nan"), dtype=torch.bfloat16, device="cuda")
+    fg.output_projection(batch, xd, wd, y)
+    torch.cuda.synchronize()
+    got = to_bits(y)
+    ref = linear(x_bits, w_bits)
+    g, r = bf16_to_f64(got), bf16_to_f64(ref)
+    absum = np.abs(bf16_to_f64(x_bits)) @ np.abs(bf16_to_f64(w_bits)).T
+    assert np.all(np.isfinite(g))
+    bound = 2.0 ** -7 * np.abs(r) + 2.0 ** -12 * absum
+    assert np.all(np.abs(g - r) <= bound), f"max excess {np.max(np.abs(g - r) - bound):.3g}"
+    assert np.mean(got != ref) < 0.01, f"{np.mean(got != ref):.3%} words differ"
+    _free(cache, batch)

@@ -227,6 +227,33 @@ def test_pass_without_rotary_appends_the_bits_and_attends_with_q_itself():
                 assert np.allclose(out[cu[s] + j, h], ref, rtol=0, atol=1e-12)
 
 
+def test_linear_against_term_by_term_sums():
+    """The output-projection oracle (a linear layer, y = o W^T) on a tiny case
+    against sums written out term by term (math.fsum, exact) and a
+    brute-force nearest-bf16 rounding; a transposed weight or a dropped term
+    changes the words."""
+    import math
+    from oracle import linear
+    from oracle.bf16 import bf16_bits_to_f64 as widen
+    rng = np.random.default_rng(6)
+    T, K, N = 4, 128, 3
+    x = f32_to_bf16_bits(rng.standard_normal((T, K)).astype(np.float32))
+    w = f32_to_bf16_bits((rng.standard_normal((N, K)) / 8).astype(np.float32))
+    y = linear(x, w)
+    assert y.shape == (T, N)
+    allv = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    fin = allv[np.isfinite(widen(allv))]
+    grid = widen(fin)
+    xs, ws = widen(x), widen(w)
+    for t in range(T):
+        for j in range(N):
+            exact = math.fsum(float(xs[t, i]) * float(ws[j, i]) for i in range(K))
+            dist = np.abs(grid - exact)
+            best = fin[dist == dist.min()]
+            want = best[0] if len(best) == 1 else best[(best & 1) == 0][0]
+            assert y[t, j] == want, (t, j)
+
+
 def test_qkv_projection_against_term_by_term_sums():
     """The projection oracle on a tiny case against sums written out term by
     term (math.fsum, exact) and a brute-force nearest-bf16 rounding."""
