@@ -81,6 +81,14 @@ fg_status fg_kv_cache_create_external(int32_t block_size, int32_t n_blocks, int3
  * (strides_elems[0] = block, [1] = K|V, [2] = head, [3] = slot, [4] = dim). */
 fg_status fg_kv_cache_layout(const fg_kv_cache* cache, void** base, int64_t strides_elems[5]);
 
+/* Builds the rotary cos/sin table for positions 0 .. max_position (at least;
+ * the table is sized in powers of two, 4096 positions or more) and the given
+ * rope_theta, on the host, and uploads it: the work the first rotary call
+ * for a position range does otherwise. A server calls it once at start-up
+ * with its longest context, so that no pass pays for it. Synchronous and
+ * allocating; a table that already covers the range is kept. */
+fg_status fg_kv_cache_prepare_rotary(fg_kv_cache* cache, double rope_theta, int32_t max_position);
+
 /* Releases the handle and (for fg_kv_cache_create) the pool. Waits for the
  * device first. NULL is accepted. */
 fg_status fg_kv_cache_destroy(fg_kv_cache* cache);

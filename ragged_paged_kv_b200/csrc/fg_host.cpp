@@ -380,6 +380,13 @@ extern "C" fg_status fg_kv_cache_layout(const fg_kv_cache* c, void** base, int64
   return FG_OK;
 }
 
+extern "C" fg_status fg_kv_cache_prepare_rotary(fg_kv_cache* c, double rope_theta, int32_t max_position) {
+  if (!c) return fail(FG_ERR_INVALID_ARG, "cache is NULL");
+  if (!(rope_theta > 0.0)) return fail(FG_ERR_INVALID_ARG, "rope_theta must be > 0");
+  if (max_position < 0) return fail(FG_ERR_INVALID_ARG, "max_position %d < 0", max_position);
+  return ensure_rope(c, rope_theta, max_position);
+}
+
 extern "C" fg_status fg_kv_cache_destroy(fg_kv_cache* c) {
   if (!c) return FG_OK;
   if (c->owned || c->rope) cudaDeviceSynchronize();

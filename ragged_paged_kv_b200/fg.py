@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
         "fg_kv_append": [V, V, V, V, V],
         "fg_qkv_rotary_kv_append": [V, V, V, V, I32, V, I32, D, V],
         "fg_output_projection": [V, V, V, I32, I32, V, V],
+        "fg_kv_cache_prepare_rotary": [V, D, I32],
         "fg_ragged_attention": [V, V, V, V, I32, F, I32, V],
         "fg_ragged_attention_noalloc": [V, V, V, V, I32, F, I32, V],
         "fg_device_status": [V, V],
@@ -158,6 +159,12 @@ class KVCache:
         strides = (ctypes.c_int64 * 5)()
         _check(lib().fg_kv_cache_layout(self._h, ctypes.byref(base), strides), "fg_kv_cache_layout")
         return base.value, list(strides)
+
+    def prepare_rotary(self, rope_theta: float, max_position: int):
+        """Build the rotary table for positions 0 .. max_position up front
+        (see fg_kv_cache_prepare_rotary)."""
+        _check(lib().fg_kv_cache_prepare_rotary(self._h, float(rope_theta), int(max_position)),
+               "fg_kv_cache_prepare_rotary")
 
     def close(self):
         if self._h:

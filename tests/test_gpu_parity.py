@@ -411,3 +411,23 @@ def test_output_projection(which):
     assert np.all(np.abs(g - r) <= bound), f"max excess {np.max(np.abs(g - r) - bound):.3g}"
     assert np.mean(got != ref) < 0.01, f"{np.mean(got != ref):.3%} words differ"
     _free(cache, batch)
+
+
+def test_prepared_rotary_table_gives_the_same_bits():
+    """fg_kv_cache_prepare_rotary builds a larger table up front (20000
+    positions -> 32768 rows): the rotated Q and the cache stay bit-exact
+    against the oracle and the outputs within tolerance."""
+    w = W.config1()
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+    fixtures.fill(cache.tensor)
+    cache.prepare_rotary(w.rope_theta, 20000)
+    cache2, batch, q_rot, out, kept = run_gpu(w, range(w.n_seqs), cache=cache)
+    pc, q_rot_ref, ref = run_oracle(w, kept)
+    assert np.array_equal(to_bits(q_rot), q_rot_ref), "rotated Q differs"
+    for s in range(w.n_seqs):
+        ids = w.block_tables[s, :w.blocks_used(s)].astype(np.int64)
+        dev = to_bits(cache.tensor[torch.from_numpy(ids).cuda()])
+        for i, b in enumerate(ids):
+            assert np.array_equal(dev[i], pc.block(int(b))), f"cache block {b} of seq {s} differs"
+    assert_close(bf16_to_f64(to_bits(out)), ref, w.name)
+    _free(cache, batch)
