@@ -1172,11 +1172,11 @@ extern "C" fg_status fg_qkv_rotary_kv_append(fg_kv_cache* c, const fg_ragged_bat
 extern "C" fg_status fg_output_projection(const fg_ragged_batch* b, const void* attn_out, const void* w_o,
                                           int32_t in_features, int32_t out_features, void* y, void* stream) {
   if (!b) return fail(FG_ERR_INVALID_ARG, "batch is NULL");
-  if (!b->cache) return fail(FG_ERR_INVALID_ARG, "batch has no valid put");
   if (in_features < 64 || in_features % 64)
     return fail(FG_ERR_UNSUPPORTED, "in_features %d is not a positive multiple of 64", in_features);
   if (out_features < 64 || out_features % 64)
     return fail(FG_ERR_UNSUPPORTED, "out_features %d is not a positive multiple of 64", out_features);
+  if (!b->cache) return fail(FG_ERR_INVALID_ARG, "batch has no valid put");
   int dev = -1;
   if (cudaGetDevice(&dev) == cudaSuccess && b->device >= 0 && dev != b->device)
     return fail(FG_ERR_INVALID_ARG, "current device %d is not the batch's device %d", dev, b->device);

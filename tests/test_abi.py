@@ -119,3 +119,25 @@ def test_host_rotary_table_equals_oracle_bitwise():
         oc, os_ = rope_table(theta, d, np.arange(p0, p0 + n))
         assert np.array_equal(c.view(np.uint32), oc.view(np.uint32))
         assert np.array_equal(s.view(np.uint32), os_.view(np.uint32))
+
+
+@pytest.mark.parametrize("k_in,n_out,status", [(4096, 4096, "FG_ERR_INVALID_ARG"),   # no put yet
+                                               (100, 4096, "FG_ERR_UNSUPPORTED"),
+                                               (4096, 96, "FG_ERR_UNSUPPORTED"),
+                                               (0, 64, "FG_ERR_UNSUPPORTED")])
+def test_output_projection_rejects_bad_arguments(k_in, n_out, status):
+    b = fg.RaggedBatch(max_tokens=8, max_seqs=2, max_blocks_per_seq=2)
+    d = ctypes.c_void_p(FAKE_DEV)
+    st = fg.lib().fg_output_projection(b.handle, d, d, k_in, n_out, d, ctypes.c_void_p(0))
+    assert fg.STATUS[st] == status
+    st = fg.lib().fg_output_projection(None, d, d, 4096, 4096, d, ctypes.c_void_p(0))
+    assert fg.STATUS[st] == "FG_ERR_INVALID_ARG"
+
+
+def test_prepare_rotary_rejects_bad_arguments():
+    h = _external()
+    L = fg.lib()
+    assert fg.STATUS[L.fg_kv_cache_prepare_rotary(h, 0.0, 100)] == "FG_ERR_INVALID_ARG"
+    assert fg.STATUS[L.fg_kv_cache_prepare_rotary(h, 10000.0, -1)] == "FG_ERR_INVALID_ARG"
+    assert fg.STATUS[L.fg_kv_cache_prepare_rotary(None, 10000.0, 100)] == "FG_ERR_INVALID_ARG"
+    L.fg_kv_cache_destroy(h)
