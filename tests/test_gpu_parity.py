@@ -431,3 +431,66 @@ def test_prepared_rotary_table_gives_the_same_bits():
             assert np.array_equal(dev[i], pc.block(int(b))), f"cache block {b} of seq {s} differs"
     assert_close(bf16_to_f64(to_bits(out)), ref, w.name)
     _free(cache, batch)
+
+
+@pytest.mark.parametrize("which", ["mha_d128", "gqa_d64", "mha_d64"])
+def test_peaked_scores_exercise_the_running_max_rescale(which):
+    """Queries scaled by 16 (exact in bf16) make the scores spread over tens
+    of log2 units, so the running maximum keeps rising by more than the
+    lazy-rescale threshold from one key tile to the next and every kernel's
+    rescale path (the O rows in TMEM or registers, the split partials, the
+    combine) runs. Rotated Q bit-exact; outputs against the oracle on the
+    same scaled queries.
+
+    With the softmax this peaked an output is close to one V row, so outputs
+    reach |V| ~ 5, where the fixed 2e-2 bound of the O(1) cases no longer
+    covers bf16 itself: rounding the exact result to bf16 alone moves it by
+    up to 2^-8 |O| (0.0156 at |O| in [4, 8)). The weights P enter the P.V
+    product rounded to bf16 (relative 2^-9 each) while their sum is kept in
+    fp32, which moves O by at most 2^-9 A, A = sum p |V| / sum p (the same
+    attention over |V|, computed by the oracle). Each output is therefore
+    held to 2e-2 + 2^-8 |O| + 2^-7 A (four times the weight term), and the
+    relative L2 error to the usual 5e-3."""
+    from oracle.bf16 import f64_to_bf16_bits
+    shapes = {"mha_d128": (32, 32, 128, 64), "gqa_d64": (8, 2, 64, 16), "mha_d64": (4, 4, 64, 16)}
+    Hq, Hkv, d, B = shapes[which]
+    w = W._make("peaked_" + which, Hq, Hkv, d, B, [0, 1, 2, 3], [300, 1, 1, 17], [0, 3000, 700, 500],
+                seed=41, budget=319)
+    q0, k, v = w.qkv()
+    q = f64_to_bf16_bits(bf16_to_f64(q0) * 16.0)
+    assert np.array_equal(bf16_to_f64(q), bf16_to_f64(q0) * 16.0)
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+    fixtures.fill(cache.tensor)
+    kept = fixtures.write_context(w, cache.tensor, set(range(w.n_seqs)))
+    batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+    batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables)
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    q_rot = torch.empty_like(qd)
+    out = torch.full_like(qd, float("nan"))
+    fg.rotary_kv_append(cache, batch, qd, kd, vd, q_rot, w.n_q_heads, w.rope_theta)
+    fg.ragged_attention(cache, batch, q_rot, out, w.n_q_heads, w.softmax_scale, w.sliding_window)
+    torch.cuda.synchronize()
+    batch.device_status()
+    pc = PagedCache(w.n_blocks, w.n_kv_heads, w.block_size, w.head_dim, fill=SENTINEL)
+    for s, (ids, blocks) in kept.items():
+        for i, b in enumerate(ids):
+            pc.blocks[int(b)] = blocks[i].copy()
+    pc_abs = PagedCache(w.n_blocks, w.n_kv_heads, w.block_size, w.head_dim, fill=SENTINEL)
+    for i, blk in pc.blocks.items():
+        a = blk.copy()
+        a[1] &= np.uint16(0x7FFF)  # |V|: clear the sign bits of the V half
+        pc_abs.blocks[i] = a
+    q_ref, _, ref = splitfuse_pass(pc, w.block_tables, w.q_lens, w.ctx_lens, q, k, v, w.rope_theta,
+                                   w.softmax_scale, w.sliding_window)
+    _, _, mass = splitfuse_pass(pc_abs, w.block_tables, w.q_lens, w.ctx_lens, q, k, v & np.uint16(0x7FFF),
+                                w.rope_theta, w.softmax_scale, w.sliding_window)
+    assert np.array_equal(to_bits(q_rot), q_ref), "rotated Q differs"
+    got = bf16_to_f64(to_bits(out))
+    assert np.isfinite(got).all()
+    err = np.abs(got - ref)
+    bound = MAX_ABS + 2.0 ** -8 * np.abs(ref) + 2.0 ** -7 * mass
+    assert np.all(err <= bound), f"{w.name}: max excess {np.max(err - bound):.3g}"
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel <= REL_L2, f"{w.name}: rel-L2 {rel:.3g}"
+    _free(cache, batch)
