@@ -254,6 +254,19 @@ def test_linear_against_term_by_term_sums():
             assert y[t, j] == want, (t, j)
 
 
+def test_linear_rounds_the_exact_sum_once():
+    """A sum whose exact value lies just above a bf16 midpoint: 1 + 2^-8 +
+    2^-40 must round up to 1 + 2^-7. A float32 sum first lands on the
+    midpoint 1 + 2^-8, and then rounds to even, down to 1. The mirror case
+    with the last term negative rounds down. Every input is a bf16 value."""
+    from oracle import linear
+    x = f32_to_bf16_bits(np.array([[1.0, 1.0, 1.0]], dtype=np.float32))
+    for tail, want in ((2.0 ** -40, 1.0 + 2.0 ** -7), (-(2.0 ** -40), 1.0)):
+        w = f32_to_bf16_bits(np.array([[1.0, 2.0 ** -8, tail]], dtype=np.float32))
+        assert bf16_bits_to_f64(linear(x, w))[0, 0] == want
+        assert bf16_bits_to_f64(linear(x, w ^ np.uint16(0x8000)))[0, 0] == -want
+
+
 def test_qkv_projection_against_term_by_term_sums():
     """The projection oracle on a tiny case against sums written out term by
     term (math.fsum, exact) and a brute-force nearest-bf16 rounding."""

@@ -141,3 +141,35 @@ def test_append_slot_off_by_one_is_caught(monkeypatch):
         return orig(self, bt_row, (np.asarray(positions) + 1) % self.block_size + 0 * np.asarray(positions), k_bits, v_bits)
     monkeypatch.setattr(opc.PagedCache, "write_positions", shifted)
     _fails(T_att.test_append_is_a_bit_copy_and_leaves_other_slots)
+
+
+# ----------------------------------------------------------- projection
+def _linear_with(mut):
+    def linear(x_bits, w_bits):
+        x = obf.bf16_bits_to_f64(np.asarray(x_bits, dtype=np.uint16))
+        w = obf.bf16_bits_to_f64(np.asarray(w_bits, dtype=np.uint16))
+        return mut(x, w)
+    return linear
+
+
+def _dropped_term(x, w):
+    return obf.f64_to_bf16_bits(x[:, :-1] @ w[:, :-1].T)
+
+
+def _through_float32(x, w):
+    return obf.f64_to_bf16_bits((x @ w.T).astype(np.float32).astype(np.float64))
+
+
+def _truncated(x, w):
+    y = (x @ w.T).astype(np.float32)
+    return (y.view(np.uint32) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("mut,pin", [(_dropped_term, "test_linear_against_term_by_term_sums"),
+                                     (_through_float32, "test_linear_rounds_the_exact_sum_once"),
+                                     (_truncated, "test_linear_against_term_by_term_sums")],
+                         ids=["dropped_term", "float32_sum", "truncation"])
+def test_linear_mistakes_are_caught(monkeypatch, mut, pin):
+    import oracle
+    monkeypatch.setattr(oracle, "linear", _linear_with(mut))
+    _fails(getattr(T_att, pin))
