@@ -277,6 +277,14 @@ def cpu_baseline(w, max_chunk_rows=4096, reps=4):
             "sample": f"{what}, float64 numpy, {len(times)} passes of {t:.2f} s"}
 
 
+def workload_config(w, ws):
+    """The `config` object both arms print: the workload, by what it is."""
+    return {"workload": f"{w.name} ({w.n_q_heads}/{w.n_kv_heads} heads, d={w.head_dim})",
+            "tokens_per_gpu": w.n_tokens, "seqs": w.n_seqs, "q_heads": w.n_q_heads,
+            "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+            "pool_blocks": w.n_blocks, "note": w.note, "parallelism": f"replicas x{ws}"}
+
+
 def run_reference(args, w, rank, ws):
     if rank != 0:
         return 0
@@ -291,9 +299,7 @@ def run_reference(args, w, rank, ws):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": w.name, "tokens": w.n_tokens, "seqs": w.n_seqs,
-                       "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
-                       "block_size": w.block_size, "note": w.note},
+            "config": workload_config(w, ws),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"{sub.n_tokens} tokens per step (all decodes + first "
                                        f"{int(sub.q_lens.max())} tokens of each chunk)"},
@@ -477,11 +483,8 @@ def run_fg(args, w, rank, ws, local_rank):
         "metric": METRIC, "value": tokens / (ms / 1000), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{w.name} ({w.n_q_heads}/{w.n_kv_heads} heads, d={w.head_dim})", "tokens_per_gpu": w.n_tokens,
-                   "seqs": w.n_seqs, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
-                   "head_dim": w.head_dim, "block_size": w.block_size, "pool_blocks": w.n_blocks,
-                   "note": w.note, "l2": "flushed between steps (256 MB write, then the same 256 MB read back; outside the events)",
-                   "parallelism": f"replicas x{ws}"},
+        "config": dict(workload_config(w, ws),
+                       l2="flushed between steps (256 MB write, then the same 256 MB read back; outside the events)"),
         "roofline": roof,
         "e2e": {"value": tokens / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
