@@ -381,9 +381,12 @@ def run_fg(args, w, rank, ws, local_rank):
         barrier()
         torch.cuda.synchronize()
         for i in range(args.steps):
-            # before the first step the flush is repeated, so that the host
-            # has its first batch put done when the device gets to the step
-            for _ in range(4 if i == 0 else 1):
+            # before the first step the flush is repeated (about 1.3 ms of
+            # device work), so that the host has validated and enqueued the
+            # first step before the device gets to it: batches of hundreds of
+            # sequences take the host about 0.6 ms, and later steps find the
+            # host ahead of the device, as in a serving loop
+            for _ in range(16 if i == 0 else 1):
                 flush_l2()
             t0 = time.perf_counter()
             step(evs[i])
