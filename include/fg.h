@@ -267,6 +267,27 @@ fg_status fg_output_projection(const fg_ragged_batch* batch, const void* attn_ou
  * info[6..7] = 0. */
 fg_status fg_attention_plan_info(const fg_ragged_batch* batch, int32_t info[8]);
 
+/* The work plan fg_ragged_attention would use for a batch of these lengths,
+ * built on the host alone (no device, no handle), for tests and tooling.
+ * q_lens / ctx_lens: host arrays of n_seqs entries (q >= 1, ctx >= 0);
+ * group = n_q_heads / n_kv_heads; head_dim 64 or 128; window 0 = none;
+ * use_tc != 0: the tensor-core kernels serve the batch (group a power of two
+ * <= 128, as fg_ragged_attention decides when the cache's tensor map can be
+ * built); slots: CTAs of the persistent query-tile kernel (the SM count).
+ * counts[0..6] = general, decode, query-tile and keys-as-rows decode units,
+ * combine groups, partial rows, largest combine row count; counts[7..10] =
+ * byte offsets of the decode, query-tile, keys-as-rows and combine lists in
+ * the packed plan (the general list starts at 0); counts[11] = packed bytes.
+ * With out != NULL and out_bytes >= counts[11] the packed plan is copied to
+ * out: lists of 32-byte units (int32 seq, kv_head, tok_begin, n_tok,
+ * key_begin, key_end, part, n_rows; part -1 = final output, else the first
+ * partial row) and 32-byte combine groups (int32 seq, kv_head, tok_begin,
+ * n_tok, part_base, n_splits, n_rows, pad); FG_ERR_CAPACITY when out_bytes
+ * is too small. */
+fg_status fg_plan_describe(const int32_t* q_lens, const int32_t* ctx_lens, int32_t n_seqs, int32_t n_kv_heads,
+                           int32_t group, int32_t head_dim, int32_t window, int32_t use_tc, int32_t slots,
+                           void* out, size_t out_bytes, int64_t counts[12]);
+
 /* Kernel timing for profiling. With `enable` != 0, each later
  * fg_ragged_attention call on this batch records CUDA events around its
  * kernels, on the streams they run on; fg_attention_kernel_ms then waits for

@@ -1018,6 +1018,38 @@ extern "C" fg_status fg_attention_plan_info(const fg_ragged_batch* b, int32_t in
   return FG_OK;
 }
 
+extern "C" fg_status fg_plan_describe(const int32_t* q_lens, const int32_t* ctx_lens, int32_t n_seqs,
+                                     int32_t n_kv_heads, int32_t group, int32_t head_dim, int32_t window,
+                                     int32_t use_tc, int32_t slots, void* out, size_t out_bytes,
+                                     int64_t counts[12]) {
+  if (n_seqs < 0 || (n_seqs > 0 && (!q_lens || !ctx_lens)) || !counts)
+    return fail(FG_ERR_INVALID_ARG, "fg_plan_describe: bad argument");
+  if (n_kv_heads < 1 || group < 1 || (head_dim != 64 && head_dim != 128) || window < 0 || slots < 1)
+    return fail(FG_ERR_INVALID_ARG, "fg_plan_describe: bad shape");
+  for (int32_t s = 0; s < n_seqs; ++s)
+    if (q_lens[s] < 1 || ctx_lens[s] < 0) return fail(FG_ERR_INVALID_ARG, "fg_plan_describe: bad lengths");
+  std::vector<int32_t> ql(q_lens, q_lens + n_seqs), cl(ctx_lens, ctx_lens + n_seqs);
+  fg::Plan P;
+  fg::build_plan(ql, cl, n_kv_heads, group, head_dim, window, use_tc != 0, slots, &P);
+  counts[0] = P.n_general;
+  counts[1] = P.n_decode;
+  counts[2] = P.n_tc;
+  counts[3] = P.n_dtc;
+  counts[4] = P.n_combine;
+  counts[5] = P.part_rows;
+  counts[6] = P.max_combine_rows;
+  counts[7] = (int64_t)P.off_decode;
+  counts[8] = (int64_t)P.off_tc;
+  counts[9] = (int64_t)P.off_dtc;
+  counts[10] = (int64_t)P.off_combine;
+  counts[11] = (int64_t)P.bytes();
+  if (out) {
+    if (out_bytes < P.bytes()) return fail(FG_ERR_CAPACITY, "plan needs %zu bytes", P.bytes());
+    P.pack(out);
+  }
+  return FG_OK;
+}
+
 extern "C" fg_status fg_device_status(fg_ragged_batch* b, void* stream) {
   if (!b) return fail(FG_ERR_INVALID_ARG, "batch is NULL");
   if (!b->derr) return FG_OK;

@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         "fg_selftest_bounded_wait": [I64, V],
         "fg_attention_kernel_ms": [V, _c_float_p],
         "fg_rotary_table": [D, I32, I32, I32, _c_float_p, _c_float_p],
+        "fg_plan_describe": [_c_int32_p, _c_int32_p, I32, I32, I32, I32, I32, I32, I32, V, SZ,
+                             ctypes.POINTER(I64)],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -315,6 +317,31 @@ def rotary_table(rope_theta: float, head_dim: int, pos_begin: int, n_pos: int):
                                  c.ctypes.data_as(_c_float_p), s.ctypes.data_as(_c_float_p)),
            "fg_rotary_table")
     return c, s
+
+
+def describe_plan(q_lens, ctx_lens, n_kv_heads: int, group: int, head_dim: int, window: int = 0,
+                  use_tc: bool = True, slots: int = 148):
+    """The attention work plan for these lengths, built on the host (see
+    fg_plan_describe): a dict of int32 arrays [n, 8] for "general",
+    "decode", "tc", "dtc" (units) and "combine" (groups), plus "part_rows"
+    and "max_combine_rows"."""
+    ql, cl = _i32(q_lens, "q_lens"), _i32(ctx_lens, "ctx_lens")
+    if ql.shape != cl.shape or ql.ndim != 1:
+        raise ValueError("q_lens and ctx_lens must be 1-d arrays of the same length")
+    counts = (ctypes.c_int64 * 12)()
+    args = (ql.ctypes.data_as(_c_int32_p), cl.ctypes.data_as(_c_int32_p), int(ql.size), int(n_kv_heads),
+            int(group), int(head_dim), int(window), int(bool(use_tc)), int(slots))
+    _check(lib().fg_plan_describe(*args, None, 0, counts), "fg_plan_describe")
+    buf = np.zeros(max(int(counts[11]), 4) // 4, dtype=np.int32)
+    _check(lib().fg_plan_describe(*args, buf.ctypes.data_as(ctypes.c_void_p), buf.nbytes, counts),
+           "fg_plan_describe")
+    offs = [0, counts[7], counts[8], counts[9], counts[10]]
+    out = {}
+    for i, name in enumerate(("general", "decode", "tc", "dtc", "combine")):
+        n = int(counts[i])
+        out[name] = buf[offs[i] // 4: offs[i] // 4 + 8 * n].reshape(n, 8).copy()
+    out["part_rows"], out["max_combine_rows"] = int(counts[5]), int(counts[6])
+    return out
 
 
 def forward(cache: KVCache, batch: RaggedBatch, q, k, v, q_rot, out, n_q_heads: int,
