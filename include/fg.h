@@ -13,6 +13,9 @@
  *      blocked as in PagedAttention),
  *   3. runs one ragged causal attention of every new token over its
  *      sequence's cached context.
+ * Around those steps it also provides the layer's Q/K/V projection fused
+ * with steps 1 and 2 (fg_qkv_rotary_kv_append) and its output projection
+ * (fg_output_projection), both on the tensor cores.
  *
  * Conventions shared by every call
  *   - Types: all tensors are bf16 (16-bit words), row-major, densely packed.
