@@ -68,6 +68,11 @@ def test_splitfuse_composer_conserves_tokens():
 def test_snapshot_is_full_and_late_enough():
     it, batch = W.splitfuse_snapshot(2, 2048, 50)
     assert it >= 50 and sum(b[1] for b in batch) == 2048
+    # and it is the first such iteration (reading c8)
+    for it2, batch2 in W.splitfuse_schedule(seed=2, budget=2048):
+        if it2 >= it:
+            break
+        assert it2 < 50 or sum(b[1] for b in batch2) < 2048
 
 
 def test_positions_not_chunking_define_token_data():
