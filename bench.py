@@ -312,67 +312,92 @@ def run_reference(args, w, rank, ws):
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
-def run_fg(args, w, rank, ws, local_rank):
-    import torch
-    from ragged_paged_kv_b200 import fg, fixtures
+class FgPass:
+    """Device state of one workload on one GPU: the cache with its prior
+    context, a batch handle, q/k/v resident in HBM and the L2 flush buffer."""
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    stream = torch.cuda.Stream(device=dev)
-    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim, device=dev)
-    fixtures.fill(cache.tensor, 0)
-    # prior context: seeded N(0,1) bf16 blocks (a pool of them, reused across
-    # sequences: same sizes and distribution, fast to set up for any pool)
-    fixtures.write_context(w, cache.tensor, keep=(), others="pool")
-    batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
-    batch.set_overlap(args.overlap)
-    q, k, v = fixtures.qkv_device(w, dev)
-    q_rot, out = torch.empty_like(q), torch.empty_like(q)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    torch.cuda.synchronize()
+    def __init__(self, w, dev, overlap=False):
+        import torch
+        from ragged_paged_kv_b200 import fg, fixtures
+        self.w, self.dev = w, dev
+        self.stream = torch.cuda.Stream(device=dev)
+        self.cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim, device=dev)
+        fixtures.fill(self.cache.tensor, 0)
+        # prior context: seeded N(0,1) bf16 blocks (a pool of them, reused
+        # across sequences: same sizes and distribution, fast for any pool)
+        fixtures.write_context(w, self.cache.tensor, keep=(), others="pool")
+        self.batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+        self.batch.set_overlap(overlap)
+        self.q, self.k, self.v = fixtures.qkv_device(w, dev)
+        self.q_rot, self.out = torch.empty_like(self.q), torch.empty_like(self.q)
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.host_parts = {"put": 0.0, "append": 0.0, "attention": 0.0}
+        torch.cuda.synchronize()
 
-    host_parts = {"put": 0.0, "append": 0.0, "attention": 0.0}
-
-    def step(ev):
-        ev[0].record(stream)
+    def step(self, ev):
+        from ragged_paged_kv_b200 import fg
+        w, st = self.w, self.stream
+        ev[0].record(st)
         t0 = time.perf_counter()
-        batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, stream)
+        self.batch.put(self.cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, st)
         t1 = time.perf_counter()
-        ev[3].record(stream)
-        fg.rotary_kv_append(cache, batch, q, k, v, q_rot, w.n_q_heads, w.rope_theta, stream)
+        ev[3].record(st)
+        fg.rotary_kv_append(self.cache, self.batch, self.q, self.k, self.v, self.q_rot, w.n_q_heads,
+                            w.rope_theta, st)
         t2 = time.perf_counter()
-        ev[1].record(stream)
-        fg.ragged_attention(cache, batch, q_rot, out, w.n_q_heads, w.softmax_scale,
-                            w.sliding_window, stream)
+        ev[1].record(st)
+        fg.ragged_attention(self.cache, self.batch, self.q_rot, self.out, w.n_q_heads, w.softmax_scale,
+                            w.sliding_window, st)
         t3 = time.perf_counter()
-        ev[2].record(stream)
-        host_parts["put"] += t1 - t0
-        host_parts["append"] += t2 - t1
-        host_parts["attention"] += t3 - t2
+        ev[2].record(st)
+        self.host_parts["put"] += t1 - t0
+        self.host_parts["append"] += t2 - t1
+        self.host_parts["attention"] += t3 - t2
 
-    def flush_l2():
+    def flush_l2(self):
         # write a buffer larger than L2 (evicts every line of the step), then
         # read it back, so that the write-back of the dirty flush lines is
         # paid here and not by the first kernel of the next step
-        with torch.cuda.stream(stream):
-            flush.zero_()
-            flush.sum()
+        import torch
+        with torch.cuda.stream(self.stream):
+            self.flush.zero_()
+            self.flush.sum()
 
-    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    for _ in range(args.warmup):
-        step(mk())
-        flush_l2()
+    def close(self):
+        import torch
+        torch.cuda.synchronize()
+        self.cache.close()
+        self.batch.close()
+        del self.cache, self.batch, self.q, self.k, self.v, self.q_rot, self.out, self.flush
+        torch.cuda.empty_cache()
+
+
+def _events():
+    import torch
+    return [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+
+def device_timing(fp, steps, warmup, local_rank):
+    """W untimed steps, then K timed steps (CUDA events on the launching
+    stream, barrier + synchronize on both sides, L2 flushed before each step
+    outside the events), with the clocks sampled during the timed region; then
+    a second pass with the library's per-kernel events. Times are the max over
+    ranks of each rank's mean."""
+    import torch
+    dev = fp.dev
+    for _ in range(warmup):
+        fp.step(_events())
+        fp.flush_l2()
     torch.cuda.synchronize()
-    batch.device_status(stream)
-
-    evs = [mk() for _ in range(args.steps)]
+    fp.batch.device_status(fp.stream)
+    evs = [_events() for _ in range(steps)]
     host_s = 0.0
-    for k_ in host_parts:
-        host_parts[k_] = 0.0
-    batch.host_profile_us(reset=True)
+    for k_ in fp.host_parts:
+        fp.host_parts[k_] = 0.0
+    fp.batch.host_profile_us(reset=True)
     # the sampler thread is started before the barrier, and every step
     # (the first included) is preceded by the L2 flush, so the device has
-    # queued work while the host enqueues a step, as it does between steps
+    # queued work while the host enqueues a step, as it does between steps;
     # a short interpreter switch interval lets the sampler thread run every
     # couple of milliseconds while the main thread enqueues
     switch = sys.getswitchinterval()
@@ -380,48 +405,117 @@ def run_fg(args, w, rank, ws, local_rank):
     with ClockSampler(local_rank) as clocks:
         barrier()
         torch.cuda.synchronize()
-        for i in range(args.steps):
+        for i in range(steps):
             # before the first step the flush is repeated (about 1.3 ms of
             # device work), so that the host has validated and enqueued the
             # first step before the device gets to it: batches of hundreds of
             # sequences take the host about 0.6 ms, and later steps find the
             # host ahead of the device, as in a serving loop
             for _ in range(16 if i == 0 else 1):
-                flush_l2()
+                fp.flush_l2()
             t0 = time.perf_counter()
-            step(evs[i])
+            fp.step(evs[i])
             host_s += time.perf_counter() - t0
         torch.cuda.synchronize()
         barrier()
     sys.setswitchinterval(switch)
-    lib_host = {k_: v_ / args.steps for k_, v_ in batch.host_profile_us(reset=True).items()}
+    lib_host = {k_: v_ / steps for k_, v_ in fp.batch.host_profile_us(reset=True).items()}
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
     put_ms = sum(e[0].elapsed_time(e[3]) for e in evs) / len(evs)
     append_ms = sum(e[3].elapsed_time(e[1]) for e in evs) / len(evs)
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    ms_local = sum(step_ms) / len(step_ms)
-    ms = max_over_ranks(ms_local, dev)
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), dev)
     attn_ms_mean = max_over_ranks(sum(attn_ms) / len(attn_ms), dev)
-    batch.device_status(stream)
-    info = batch.plan_info()
+    fp.batch.device_status(fp.stream)
+    info = fp.batch.plan_info()
+    host_parts = {k_: 1000 * v_ / steps for k_, v_ in fp.host_parts.items()}
 
     # per-kernel durations: the library's own CUDA events around each kernel,
     # on the stream it runs on (a separate pass, synchronised per step so
     # the events of every step can be read; the kernels run exactly as above)
-    batch.set_timing(True)
+    fp.batch.set_timing(True)
     kms = []
-    for _ in range(args.steps):
-        step(mk())
-        kms.append(batch.kernel_ms())
-        flush_l2()
-    batch.set_timing(False)
+    for _ in range(steps):
+        fp.step(_events())
+        kms.append(fp.batch.kernel_ms())
+        fp.flush_l2()
+    fp.batch.set_timing(False)
     torch.cuda.synchronize()
     kernel_ms = {k: max_over_ranks(sum(d[k] for d in kms) / len(kms), dev) for k in kms[0]}
+    return {"ms": ms, "attn_ms": attn_ms_mean, "put_ms": put_ms, "append_ms": append_ms,
+            "kernel_ms": kernel_ms, "host_s": host_s, "host_parts": host_parts, "lib_host": lib_host,
+            "info": info, "clocks": clocks.summary()}
+
+
+def roofline_of(w, config, m):
+    """The `roofline` object for the dominant kernel of workload w (the one
+    with the longest average launch), from the measurements `m`."""
+    work = algorithmic_work(w)
+    hbm, tf, src = load_peaks()
+    kernel_ms = m["kernel_ms"]
+    dom = max(("decode", "tc"), key=lambda k: kernel_ms[k])
+    if dom == "decode":
+        achieved = work["decode_bytes"] / (kernel_ms["decode"] / 1000) / 1e9
+        roof = {"kernel": "decode (attn_decode_tc_kernel at d=128, attn_decode_kernel at d=64)", "bound": "hbm",
+                "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": ncu_traffic(config, "decode"), "algorithmic_bytes": work["decode_bytes"]}
+    elif work["tc_flops"] / (tf * 1e12) >= work["tc_bytes"] / (hbm * 1e9):
+        achieved = work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12
+        roof = {"kernel": "attn_tc_kernel (tcgen05 tiles)", "bound": "tensor", "achieved": achieved,
+                "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf, "traffic": ncu_traffic(config, "tc"),
+                "algorithmic_flops": work["tc_flops"]}
+    else:  # its tiles are mostly grouped-query decodes: bound by the K/V bytes
+        achieved = work["tc_bytes"] / (kernel_ms["tc"] / 1000) / 1e9
+        roof = {"kernel": "attn_tc_kernel (tcgen05 tiles)", "bound": "hbm", "achieved": achieved,
+                "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": ncu_traffic(config, "tc"),
+                "algorithmic_bytes": work["tc_bytes"]}
+    roof.update({"peak_source": f"{src} (MEASURED_PEAKS.json)" if src == "measured" else src,
+                 "kernel_ms": kernel_ms,
+                 "tc_TFLOPs": work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12 if kernel_ms["tc"] else None,
+                 "step_roofline_ms": 1000 * max((work["attn_bytes"] + work["append_bytes"]) / (hbm * 1e9),
+                                                work["flops"] / (tf * 1e12))})
+    roof["step_frac"] = roof["step_roofline_ms"] / m["ms"]
+    return roof
+
+
+def make_workload(config, compact_pool=False, local_rank=0, gpu=True):
+    """Workload `config`; config 3's pool fills the GPU's free memory up to
+    180 GB (less 8 GiB of headroom) when it runs on a GPU."""
+    from ragged_paged_kv_b200 import workloads as W
+    if config == 3 and gpu:
+        import torch
+        free, _ = torch.cuda.mem_get_info(local_rank)
+        w = W.config3(n_blocks=int(min(180 * 10**9, free - 8 * 2**30) // (2 * 32 * 64 * 128 * 2)))
+    else:
+        w = W.CONFIGS[config]()
+    if compact_pool:
+        need = sum(w.blocks_used(s) for s in range(w.n_seqs))
+        w = W._make(w.name, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.seq_ids,
+                    w.q_lens, w.ctx_lens, w.seed, w.budget, n_blocks=need + 16,
+                    window=w.sliding_window, note=w.note + "; compact pool")
+    return w
+
+
+# gates of the five configurations (BASELINE.md's table): the dominant
+# kernel's fraction of its roofline
+GATES = {2: ("hbm", 0.70), 3: ("hbm", 0.70), 4: ("hbm", 0.70), 5: ("tensor", 0.50)}
+
+
+def run_fg(args, w, rank, ws, local_rank):
+    import torch
+    from ragged_paged_kv_b200 import fg
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    fp = FgPass(w, dev, args.overlap)
+    m = device_timing(fp, args.steps, args.warmup, local_rank)
+    ms = m["ms"]
 
     # end to end through the public API from pinned host buffers
-    host_in = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v))}
-    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dev_bufs = {"q": q, "k": k, "v": v, "q_rot": q_rot, "out": out}
+    stream, batch, cache = fp.stream, fp.batch, fp.cache
+    host_in = {n: t.cpu().pin_memory() for n, t in (("q", fp.q), ("k", fp.k), ("v", fp.v))}
+    host_out = torch.empty(fp.out.shape, dtype=fp.out.dtype).pin_memory()
+    dev_bufs = {"q": fp.q, "k": fp.k, "v": fp.v, "q_rot": fp.q_rot, "out": fp.out}
 
     def e2e_step():
         batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, stream)
@@ -430,15 +524,15 @@ def run_fg(args, w, rank, ws, local_rank):
 
     for _ in range(max(3, args.warmup)):
         e2e_step()
-        flush_l2()
+        fp.flush_l2()
     torch.cuda.synchronize()
-    e2e_ev = [mk() for _ in range(args.steps)]
+    e2e_ev = [_events() for _ in range(args.steps)]
     barrier()
     for i in range(args.steps):
         e2e_ev[i][0].record(stream)
         e2e_step()
         e2e_ev[i][1].record(stream)
-        flush_l2()
+        fp.flush_l2()
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / args.steps, dev)
@@ -446,55 +540,67 @@ def run_fg(args, w, rank, ws, local_rank):
                       sum(w.blocks_used(s) for s in range(w.n_seqs)))
     h2d = sum(t.numel() * 2 for t in host_in.values()) + meta_bytes
     d2h = host_out.numel() * 2
+    del host_in, host_out, dev_bufs
+    fp.close()
+
+    # the other gated configurations, measured the same way in this run
+    # (fewer steps), one object each under "per_config"
+    per_config = {}
+    launches = args.steps * (1 + m["info"]["launches"])
+    if not args.no_per_config:
+        for c in sorted(GATES):
+            if c == args.config:
+                continue
+            wc = make_workload(c, args.compact_pool, local_rank)
+            fpc = FgPass(wc, dev, args.overlap)
+            mc = device_timing(fpc, args.per_config_steps, 3, local_rank)
+            fpc.close()
+            rc = roofline_of(wc, c, mc)
+            bound, gate = GATES[c]
+            per_config[str(c)] = {
+                "workload": f"{wc.name} ({wc.n_q_heads}/{wc.n_kv_heads} heads, d={wc.head_dim}, "
+                            f"{wc.n_tokens} tokens, {wc.n_seqs} seqs, pool {wc.n_blocks} blocks)",
+                "steps": args.per_config_steps, "warmup": 3, "ms_per_step": mc["ms"],
+                "tokens_per_s": wc.n_tokens * ws / (mc["ms"] / 1000),
+                "put_ms": mc["put_ms"], "append_ms": mc["append_ms"], "attention_call_ms": mc["attn_ms"],
+                "dominant_kernel": rc["kernel"], "bound": rc["bound"], "achieved": rc["achieved"],
+                "unit": rc["unit"], "peak": rc["peak"], "frac": rc["frac"], "traffic": rc["traffic"],
+                "kernel_ms": rc["kernel_ms"], "tc_TFLOPs": rc["tc_TFLOPs"],
+                "step_roofline_ms": rc["step_roofline_ms"], "step_frac": rc["step_frac"],
+                "gate": {"bound": bound, "min_frac": gate, "met": rc["bound"] == bound and rc["frac"] >= gate},
+                "clocks": mc["clocks"]}
+            launches += args.per_config_steps * (1 + mc["info"]["launches"])
 
     if rank != 0:
         return 0
-    work = algorithmic_work(w)
-    hbm, tf, src = load_peaks()
     tokens = w.n_tokens * ws
-    # roofline of the dominant kernel (longest average launch)
-    dom = max(("decode", "tc"), key=lambda k: kernel_ms[k])
-    if dom == "decode":
-        achieved = work["decode_bytes"] / (kernel_ms["decode"] / 1000) / 1e9
-        roof = {"kernel": "decode (attn_decode_tc_kernel at d=128, attn_decode_kernel at d=64)", "bound": "hbm",
-                "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": ncu_traffic(args.config, "decode"), "algorithmic_bytes": work["decode_bytes"]}
-    elif work["tc_flops"] / (tf * 1e12) >= work["tc_bytes"] / (hbm * 1e9):
-        achieved = work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12
-        roof = {"kernel": "attn_tc_kernel (tcgen05 tiles)", "bound": "tensor", "achieved": achieved,
-                "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf, "traffic": ncu_traffic(args.config, "tc"),
-                "algorithmic_flops": work["tc_flops"]}
-    else:  # its tiles are mostly grouped-query decodes: bound by the K/V bytes
-        achieved = work["tc_bytes"] / (kernel_ms["tc"] / 1000) / 1e9
-        roof = {"kernel": "attn_tc_kernel (tcgen05 tiles)", "bound": "hbm", "achieved": achieved,
-                "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": ncu_traffic(args.config, "tc"),
-                "algorithmic_bytes": work["tc_bytes"]}
-    roof.update({"peak_source": f"{src} (MEASURED_PEAKS.json)" if src == "measured" else src,
-                 "kernel_ms": kernel_ms,
-                 "attention_call_ms": attn_ms_mean,
-                 "put_ms": put_ms,
-                 "append_ms": append_ms,
-                 "host_enqueue_ms_per_step": 1000 * host_s / args.steps,
-                 "host_ms_per_call": {k_: 1000 * v_ / args.steps for k_, v_ in host_parts.items()},
-                 "library_host_us_per_step": lib_host,
-                 "attention_call_GBps": work["attn_bytes"] / (attn_ms_mean / 1000) / 1e9,
-                 "tc_TFLOPs": work["tc_flops"] / (kernel_ms["tc"] / 1000) / 1e12 if kernel_ms["tc"] else None,
-                 "step_roofline_ms": 1000 * max((work["attn_bytes"] + work["append_bytes"]) / (hbm * 1e9),
-                                                work["flops"] / (tf * 1e12))})
-    roof["step_frac"] = roof["step_roofline_ms"] / ms
+    roof = roofline_of(w, args.config, m)
+    work = algorithmic_work(w)
+    roof.update({"attention_call_ms": m["attn_ms"],
+                 "put_ms": m["put_ms"],
+                 "append_ms": m["append_ms"],
+                 "host_enqueue_ms_per_step": 1000 * m["host_s"] / args.steps,
+                 "host_ms_per_call": m["host_parts"],
+                 "library_host_us_per_step": m["lib_host"],
+                 "attention_call_GBps": work["attn_bytes"] / (m["attn_ms"] / 1000) / 1e9})
+    gb, gf = GATES.get(args.config, (None, None))
+    if gb is not None:
+        roof["gate"] = {"bound": gb, "min_frac": gf, "met": roof["bound"] == gb and roof["frac"] >= gf}
     line = {
         "metric": METRIC, "value": tokens / (ms / 1000), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(w, ws),
-                       l2="flushed between steps (256 MB write, then the same 256 MB read back; outside the events)"),
+        "config": workload_config(w, ws),
+        "l2": "flushed between steps (256 MB write, then the same 256 MB read back; outside the events)",
         "roofline": roof,
         "e2e": {"value": tokens / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * (1 + info["launches"]),
-        "plan": dict(info, overlap=args.overlap),
-        "clocks": clocks.summary(),
+        "gpu_launches": launches,
+        "plan": dict(m["info"], overlap=args.overlap),
+        "clocks": m["clocks"],
     }
+    if per_config:
+        line["per_config"] = per_config
     if ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
@@ -663,7 +769,7 @@ class BlockAllocator:
         self.free.extend(self.owned.pop(rid, []))
 
 
-def run_serve_sim(args):
+def run_serve_sim(args, policy="greedy"):
     """A timed Dynamic SplitFuse loop with attention only (no weights): the
     composer's closed loop of synthetic clients (32 active of 512 requests,
     prompt ~N(2600, 30 %), output ~N(60, 30 %), budget 2048: the card's
@@ -676,7 +782,10 @@ def run_serve_sim(args):
     and one more at the end of every later iteration. One JSON line (kind
     "serve_sim"): throughput, percentiles of time to first token and of the
     mean time per output token, and the requests per second that meet the
-    latency targets (--sla-ttft-ms, --sla-tpot-ms)."""
+    latency targets (--sla-ttft-ms, --sla-tpot-ms). `policy` is the
+    composer's chunking policy ("greedy": every pass filled while prompt
+    tokens are pending; "equal_split": the pending prompt tokens spread evenly
+    over the passes they need)."""
     import torch
     from ragged_paged_kv_b200 import fg, workloads as W
     dev = torch.device("cuda", 0)
@@ -718,7 +827,7 @@ def run_serve_sim(args):
         return T, e0.elapsed_time(e1)
 
     warm_alloc = BlockAllocator(n_blocks, B, seed=1)
-    for it, bt in W.splitfuse_schedule(seed=2, budget=budget):
+    for it, bt in W.splitfuse_schedule(seed=2, budget=budget, policy=policy):
         if it >= 64:
             break
         one_pass(bt, warm_alloc)
@@ -730,6 +839,7 @@ def run_serve_sim(args):
     clock = 0.0
     iters = tokens = 0
     seen = 0
+    pass_ms, pass_tokens = [], []
 
     def settle():
         # the composer reports an iteration's outcome when it is resumed for
@@ -748,9 +858,11 @@ def run_serve_sim(args):
                 arrive[r] = clock
         seen = len(events)
 
-    for it, bt in W.splitfuse_schedule(seed=2, budget=budget, events=events):
+    for it, bt in W.splitfuse_schedule(seed=2, budget=budget, events=events, policy=policy):
         settle()
         T, ms = one_pass(bt, alloc)
+        pass_ms.append(ms)
+        pass_tokens.append(T)
         clock += ms
         iters += 1
         tokens += T
@@ -763,11 +875,14 @@ def run_serve_sim(args):
              (n_out[r] <= 1 or (last[r] - first[r]) / (n_out[r] - 1) <= args.sla_tpot_ms)]
     pct = lambda a, p: float(np.percentile(a, p)) if len(a) else None
     print(json.dumps({
-        "kind": "serve_sim", "workload": "Llama-2-7B attention shape, 32 active of 512 requests, budget 2048",
+        "kind": "serve_sim", "policy": policy,
+        "workload": "Llama-2-7B attention shape, 32 active of 512 requests, budget 2048",
         "iterations": iters, "tokens": tokens, "requests": len(done), "device_s": clock / 1e3,
         "tokens_per_s": tokens / clock * 1e3, "requests_per_s": len(done) / clock * 1e3,
         "ttft_ms": {"p50": pct(ttft, 50), "p95": pct(ttft, 95)},
         "tpot_ms": {"p50": pct(tpot, 50), "p95": pct(tpot, 95)},
+        "pass_ms": {"p50": pct(pass_ms, 50), "p95": pct(pass_ms, 95), "max": max(pass_ms)},
+        "pass_tokens": {"p50": pct(pass_tokens, 50), "min": min(pass_tokens), "max": max(pass_tokens)},
         "sla": {"ttft_ms": args.sla_ttft_ms, "tpot_ms": args.sla_tpot_ms,
                 "effective_requests_per_s": len(meets) / clock * 1e3}}), flush=True)
     return 0
@@ -781,6 +896,9 @@ def main():
     ap.add_argument("--impl", choices=["fg", "reference"], default="fg")
     ap.add_argument("--config", type=int, default=2, help="workload number (2 = the headline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="measure only the chosen config (no per_config object for the other gated configs)")
+    ap.add_argument("--per-config-steps", type=int, default=5)
     ap.add_argument("--overlap", action="store_true",
                     help="run the query-tile kernel beside the decode kernel on a second stream")
     ap.add_argument("--compact-pool", action="store_true",
@@ -789,6 +907,8 @@ def main():
                     help="time the fused Q/K/V projection + rotary + append and the output projection (one GPU; JSON lines, no contract line)")
     ap.add_argument("--serve-sim", action="store_true",
                     help="timed SplitFuse loop with closed-loop synthetic clients (one GPU; JSON line)")
+    ap.add_argument("--policy", choices=["greedy", "equal_split", "both"], default="both",
+                    help="--serve-sim: the composer's chunking policy (both: one line each)")
     ap.add_argument("--sla-ttft-ms", type=float, default=30.0)
     ap.add_argument("--sla-tpot-ms", type=float, default=1.0)
     ap.add_argument("--sweep-tokens", action="store_true",
@@ -799,19 +919,13 @@ def main():
     if args.sweep_tokens:
         return run_token_sweep(args)
     if args.serve_sim:
-        return run_serve_sim(args)
-    from ragged_paged_kv_b200 import workloads as W
-    if args.config == 3 and args.impl == "fg":
-        import torch
-        free, _ = torch.cuda.mem_get_info(world()[2])
-        w = W.config3(n_blocks=int(min(180 * 10**9, free - 8 * 2**30) // (2 * 32 * 64 * 128 * 2)))
-    else:
-        w = W.CONFIGS[args.config]()
-    if args.compact_pool:
-        need = sum(w.blocks_used(s) for s in range(w.n_seqs))
-        w = W._make(w.name, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size, w.seq_ids,
-                    w.q_lens, w.ctx_lens, w.seed, w.budget, n_blocks=need + 16,
-                    window=w.sliding_window, note=w.note + "; compact pool")
+        from ragged_paged_kv_b200 import workloads as W
+        for pol in (W.POLICIES if args.policy == "both" else (args.policy,)):
+            rc = run_serve_sim(args, pol)
+            if rc:
+                return rc
+        return 0
+    w = make_workload(args.config, args.compact_pool, world()[2], gpu=args.impl == "fg")
     if args.qkv_fused:
         return run_qkv_fused(args, w)
     if args.impl == "reference":

@@ -285,18 +285,18 @@ cudaError_t launch_decode_d(const CacheView& cache, const BatchView& batch, cons
                             float* part_o, float* part_ml, int Hq, float scale_log2,
                             cudaStream_t stream) {
   using C = DecodeCfg<D>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
+  // per device: the attributes apply to the current device only
+  static PerDeviceOnce configured;
+  cudaError_t e0 = configured.run([] {
+    cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     // the largest shared-memory carveout, so CTAs of different kernels can
     // share an SM
-    e = cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    return e;
+  });
+  if (e0 != cudaSuccess) return e0;
   attn_decode_kernel<D><<<n_items, C::kThreads, C::kSmem, stream>>>(cache, batch, items, q_rot, out,
                                                                     part_o, part_ml, Hq, scale_log2);
   return cudaGetLastError();

@@ -475,18 +475,18 @@ cudaError_t launch_attention_decode_tc(const void* tm_q1, const void* tm_kv, con
                                        int sm_tc_end, const int* tc_counter, int n_tc, bool pdl,
                                        cudaStream_t stream) {
   if (n_items == 0) return cudaSuccess;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         DtcCfg::kSmem);
-    if (e != cudaSuccess) return e;
+  // per device: the attributes apply to the current device only
+  static PerDeviceOnce configured;
+  cudaError_t e0 = configured.run([] {
+    cudaError_t e = cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DtcCfg::kSmem);
     // the largest shared-memory carveout, so CTAs of different kernels can
     // share an SM
-    e = cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    return e;
+  });
+  if (e0 != cudaSuccess) return e0;
   DtcArgs args{cache, batch, items, out, part_o, part_ml, n_q_heads, g, scale_log2, n_items, counter,
                sm_tc_end, tc_counter, n_tc};
   grid = grid < 1 ? 1 : (grid > n_items ? n_items : grid);

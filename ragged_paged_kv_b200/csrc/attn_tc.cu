@@ -599,16 +599,18 @@ template <int D>
 cudaError_t launch_tc_d(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const TcArgs& args, int grid,
                         cudaStream_t stream) {
   using C = TcCfg<D>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e =
-        cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // per device: the attributes apply to the current device only
+  static PerDeviceOnce configured;
+  cudaError_t e0 = configured.run([] {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    // the largest shared-memory carveout, so CTAs of different kernels can
+    // share an SM
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+    return e;
+  });
+  if (e0 != cudaSuccess) return e0;
   attn_tc_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tm_q, tm_kv, args);
   return cudaGetLastError();
 }

@@ -831,25 +831,40 @@ fg_status ensure_workspace(fg_ragged_batch* b, size_t floats, cudaStream_t strm)
 
 }  // namespace
 
-fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot,
-                              void* out, int32_t n_q_heads, float softmax_scale,
-                              int32_t window, cudaStream_t strm, float* ws, size_t ws_floats,
-                              bool grow_ws);
+// Where an attention pass keeps its split workspace and its work plan when
+// the caller supplies them (the allocation-free entry point): `ws` holds
+// ws_floats floats, `plan_dev` plan_bytes bytes whose last 256 bytes hold the
+// persistent kernels' unit counters.
+struct FixedPassStorage {
+  float* ws;
+  size_t ws_floats;
+  void* plan_dev;
+  size_t plan_bytes;
+};
+
+fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot, void* out,
+                              int32_t n_q_heads, float softmax_scale, int32_t window, cudaStream_t strm,
+                              const FixedPassStorage* fixed);
 
 extern "C" fg_status fg_ragged_attention(const fg_kv_cache* c, fg_ragged_batch* b,
                                          const void* q_rot, void* out, int32_t n_q_heads,
                                          float softmax_scale, int32_t sliding_window,
                                          void* stream) {
   return fg_attention_launch(c, b, q_rot, out, n_q_heads, softmax_scale, sliding_window,
-                             static_cast<cudaStream_t>(stream), nullptr, 0, true);
+                             static_cast<cudaStream_t>(stream), nullptr);
 }
 
-// Shared body of the attention entry points. With grow_ws the batch's own
-// workspace is used (and grown); otherwise `ws` / `ws_floats` is.
-fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot,
-                              void* out, int32_t n_q_heads, float softmax_scale,
-                              int32_t window, cudaStream_t strm, float* ws, size_t ws_floats,
-                              bool grow_ws) {
+// The one launch sequence of both attention entry points. With fixed ==
+// nullptr the batch's own workspace and double-buffered plan are used (grown
+// with stream-ordered allocation, the plan uploaded from pinned staging on
+// the copy stream and cached per batch and shape). Otherwise the plan is
+// built into thread-local host memory, sent into fixed->plan_dev with a
+// plain copy on `strm`, and the workspace is fixed->ws: nothing is allocated,
+// and the batch's own plan cache and workspace are left alone. Only the
+// storage differs; the kernels, their order and their arguments are the same.
+fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot, void* out,
+                              int32_t n_q_heads, float softmax_scale, int32_t window, cudaStream_t strm,
+                              const FixedPassStorage* fixed) {
   fg_status st = check_pass(c, b, n_q_heads);
   if (st) return st;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
@@ -869,24 +884,45 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
                  !make_q_map(&tm_q1, q_rot, b->n_tokens, n_q_heads, c->head_dim, g, 1)))
     return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q_rot");
   b->hprof[6] += now_us() - t_a;
-  st = prepare_plan(b, c, g, window, use_tc, strm);
-  const double t_l = now_us();
-  if (st) return st;
-  const fg::Plan& P = b->plan;
-  const size_t need = (size_t)P.part_rows * (c->head_dim + 2);
-  if (grow_ws) {
-    st = ensure_workspace(b, need, strm);
+  const fg::Plan* plan = &b->plan;
+  const char* base = nullptr;
+  int* ctr = nullptr;  // the persistent kernels' unit counters (zero at launch)
+  float* ws = nullptr;
+  if (!fixed) {
+    st = prepare_plan(b, c, g, window, use_tc, strm);
+    if (st) return st;
+    base = static_cast<const char*>(b->dplan.current());
+    ctr = reinterpret_cast<int*>(static_cast<char*>(b->dplan.current()) + plan->bytes());
+    st = ensure_workspace(b, (size_t)plan->part_rows * (c->head_dim + 2), strm);
     if (st) return st;
     ws = b->ws;
-  } else if (need > ws_floats) {
-    return fail(FG_ERR_CAPACITY, "pass needs %zu workspace floats, %zu available", need, ws_floats);
+  } else {
+    thread_local fg::Plan P_fixed;
+    thread_local std::vector<unsigned char> packed;
+    fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc, sm_count(), &P_fixed);
+    plan = &P_fixed;
+    if (P_fixed.bytes() + 256 > fixed->plan_bytes)
+      return fail(FG_ERR_CAPACITY, "pass needs a %zu-byte work plan, the fixed area holds %zu", P_fixed.bytes(),
+                  fixed->plan_bytes - 256);
+    const size_t need = (size_t)P_fixed.part_rows * (c->head_dim + 2);
+    if (need > fixed->ws_floats)
+      return fail(FG_ERR_CAPACITY, "pass needs %zu split-workspace floats, the fixed area holds %zu", need,
+                  fixed->ws_floats);
+    packed.resize(P_fixed.bytes());
+    P_fixed.pack(packed.data());
+    if (!packed.empty())
+      FG_CUDA(cudaMemcpyAsync(fixed->plan_dev, packed.data(), packed.size(), cudaMemcpyHostToDevice, strm));
+    base = static_cast<const char*>(fixed->plan_dev);
+    ctr = reinterpret_cast<int*>(static_cast<char*>(fixed->plan_dev) + fixed->plan_bytes - 256);
+    ws = fixed->ws;
   }
+  const fg::Plan& P = *plan;
+  const double t_l = now_us();
   float* part_o = ws;
   float* part_ml = ws ? ws + (size_t)P.part_rows * c->head_dim : nullptr;
   const float scale_log2 = softmax_scale * 1.4426950408889634f;
   b->last_launches = (P.n_general > 0) + (P.n_decode > 0) + (P.n_tc > 0) + (P.n_dtc > 0) +
                      (P.n_combine > 0);
-  const char* base = static_cast<const char*>(b->dplan.current());
   const CacheView cv = cache_view(c);
   const auto* qr = static_cast<const __nv_bfloat16*>(q_rot);
   auto* o = static_cast<__nv_bfloat16*>(out);
@@ -908,7 +944,7 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   // tensor-core tiles and MHA decode units touch disjoint outputs and
   // partial rows: run them side by side (tc on a high-priority second
   // stream forked from and joined back into the caller's stream)
-  const int tc_sms = b->overlap ? tc_share(P, c->head_dim, sm_count()) : 0;
+  const int tc_sms = b->overlap && !fixed ? tc_share(P, c->head_dim, sm_count()) : 0;
   const bool both = tc_sms > 0;
   cudaStream_t tc_stream = strm;
   if (both) {
@@ -916,10 +952,10 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
     if (st) return st;
     tc_stream = b->aux;
   }
-  // the persistent kernels' unit counters start at zero
-  int* ctr = reinterpret_cast<int*>(static_cast<char*>(b->dplan.current()) + P.bytes());
-  if ((P.n_tc || P.n_dtc) && !b->ctr_fresh) FG_CUDA(cudaMemsetAsync(ctr, 0, 8, strm));
-  b->ctr_fresh = false;
+  // the persistent kernels' unit counters start at zero (a fresh upload of
+  // the batch's own plan zeroed them already)
+  if ((P.n_tc || P.n_dtc) && (fixed || !b->ctr_fresh)) FG_CUDA(cudaMemsetAsync(ctr, 0, 8, strm));
+  if (!fixed) b->ctr_fresh = false;
   // programmatic dependent launch along the chain query tiles -> decode ->
   // combine when the kernels follow each other on one stream with nothing
   // in between (the decode kernel waits for the query-tile grid before its
@@ -1081,83 +1117,13 @@ extern "C" const char* fg_status_string(fg_status s) {
 
 extern "C" const char* fg_last_error(void) { return g_last_error.c_str(); }
 
-// Attention pass on caller-provided device storage: the split workspace is
-// `ws` (ws_floats floats) and the work plan is uploaded into `plan_dev`
-// (plan_bytes bytes) with a plain copy from host memory. Nothing is
-// allocated on the device or pinned on the host. The batch's own plan cache
-// and workspace are left alone.
+// The allocation-free entry point's launch (its storage is in attn_noalloc.cu).
 fg_status fg_attention_launch_fixed(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot,
                                     void* out, int32_t n_q_heads, float softmax_scale,
                                     int32_t window, cudaStream_t strm, float* ws,
                                     size_t ws_floats, void* plan_dev, size_t plan_bytes) {
-  fg_status st = check_pass(c, b, n_q_heads);
-  if (st) return st;
-  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-    return fail(FG_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
-  if (window < 0) return fail(FG_ERR_INVALID_ARG, "sliding_window %d < 0", window);
-  if (b->n_tokens == 0) return FG_OK;
-  if (!q_rot || !out) return fail(FG_ERR_INVALID_ARG, "NULL tensor pointer");
-  if (!aligned16(q_rot) || !aligned16(out))
-    return fail(FG_ERR_INVALID_ARG, "q_rot and out must be 16-byte aligned");
-  const int32_t g = n_q_heads / c->n_kv_heads;
-  const bool use_tc = tc_eligible(const_cast<fg_kv_cache*>(c), g);
-  if (!use_tc && g > fg::kMaxGroup)
-    return fail(FG_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads = %d > %d", g, fg::kMaxGroup);
-  CUtensorMap tm_q, tm_q1;
-  if (use_tc && (!make_q_map(&tm_q, q_rot, b->n_tokens, n_q_heads, c->head_dim, g) ||
-                 !make_q_map(&tm_q1, q_rot, b->n_tokens, n_q_heads, c->head_dim, g, 1)))
-    return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q_rot");
-  thread_local fg::Plan P;
-  thread_local std::vector<unsigned char> packed;
-  fg::build_plan(b->q_lens, b->ctx_lens, c->n_kv_heads, g, c->head_dim, window, use_tc,
-                 sm_count(), &P);
-  // the last 256 bytes of the plan area hold the persistent kernels' counters
-  if (P.bytes() + 256 > plan_bytes)
-    return fail(FG_ERR_CAPACITY, "pass needs a %zu-byte work plan, the fixed area holds %zu",
-                P.bytes(), plan_bytes - 256);
-  int* ctr = reinterpret_cast<int*>(static_cast<char*>(plan_dev) + plan_bytes - 256);
-  const size_t need = (size_t)P.part_rows * (c->head_dim + 2);
-  if (need > ws_floats)
-    return fail(FG_ERR_CAPACITY, "pass needs %zu split-workspace floats, the fixed area holds %zu",
-                need, ws_floats);
-  packed.resize(P.bytes());
-  P.pack(packed.data());
-  if (!packed.empty())
-    FG_CUDA(cudaMemcpyAsync(plan_dev, packed.data(), packed.size(), cudaMemcpyHostToDevice, strm));
-  if (P.n_tc || P.n_dtc) FG_CUDA(cudaMemsetAsync(ctr, 0, 8, strm));
-  float* part_o = ws;
-  float* part_ml = ws + (size_t)P.part_rows * c->head_dim;
-  const float scale_log2 = softmax_scale * 1.4426950408889634f;
-  const char* base = static_cast<const char*>(plan_dev);
-  const CacheView cv = cache_view(c);
-  const auto* qr = static_cast<const __nv_bfloat16*>(q_rot);
-  auto* o = static_cast<__nv_bfloat16*>(out);
-  cudaError_t e = fg::launch_attention_general(
-      cv, b->view, reinterpret_cast<const WorkItem*>(base + P.off_general), P.n_general, qr, o,
-      part_o, part_ml, n_q_heads, g, scale_log2, window, strm);
-  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-  e = fg::launch_attention_decode(cv, b->view, reinterpret_cast<const WorkItem*>(base + P.off_decode),
-                                  P.n_decode, qr, o, part_o, part_ml, n_q_heads, scale_log2, strm);
-  if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
-  if (P.n_tc) {
-    e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
-                                reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
-                                part_ml, n_q_heads, g, scale_log2, window, sm_count(), INT32_MAX,
-                                ctr, strm);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
-  }
-  if (P.n_dtc) {
-    e = fg::launch_attention_decode_tc(&tm_q1, &c->tm_kv, cv, b->view,
-                                       reinterpret_cast<const WorkItem*>(base + P.off_dtc), P.n_dtc, o,
-                                       part_o, part_ml, n_q_heads, g, scale_log2, 2 * sm_count(), ctr + 1,
-                                       0, nullptr, 0, P.n_tc > 0, strm);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core decode launch");
-  }
-  e = fg::launch_combine(b->view, reinterpret_cast<const CombineItem*>(base + P.off_combine),
-                         P.n_combine, P.max_combine_rows, part_o, part_ml, o, n_q_heads, g,
-                         c->head_dim, P.n_dtc > 0, strm);
-  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
-  return FG_OK;
+  const FixedPassStorage fixed{ws, ws_floats, plan_dev, plan_bytes};
+  return fg_attention_launch(c, b, q_rot, out, n_q_heads, softmax_scale, window, strm, &fixed);
 }
 
 // 2-D bf16 view (inner dim `inner`, outer dim `outer`, row stride inner * 2 B)

@@ -4,9 +4,31 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 namespace fg {
+
+// One-time launch set-up (cudaFuncSetAttribute and the like) per device:
+// such attributes apply to the device that is current when they are set, so
+// a process that drives several GPUs must set them on each. run(f) calls f
+// with the device current unless it already succeeded there; an ordinal
+// beyond the table runs f every time.
+struct PerDeviceOnce {
+  static constexpr int kMaxDevices = 64;
+  std::atomic<bool> done[kMaxDevices];
+  template <class F>
+  cudaError_t run(F&& f) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return f();
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = f();
+    if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+    return e;
+  }
+};
 
 // Device error word bits (read back by fg_device_status).
 enum : int32_t { kErrBadBlock = 1, kErrBadIndex = 2, kErrTimeout = 4 };

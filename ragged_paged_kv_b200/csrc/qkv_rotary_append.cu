@@ -236,13 +236,13 @@ template <int D, bool LINEAR>
 cudaError_t launch_qkv_d(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const QkvArgs& args,
                          int n_heads_total, cudaStream_t stream) {
   using C = QkvCfg<D>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(qkv_rotary_append_kernel<D, LINEAR>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // per device: the attributes apply to the current device only
+  static PerDeviceOnce configured;
+  cudaError_t e0 = configured.run([] {
+    cudaError_t e = cudaFuncSetAttribute(qkv_rotary_append_kernel<D, LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    return e;
+  });
+  if (e0 != cudaSuccess) return e0;
   dim3 grid((args.batch.n_tokens + C::BM - 1) / C::BM, n_heads_total);
   qkv_rotary_append_kernel<D, LINEAR><<<grid, C::kThreads, C::kSmem, stream>>>(tm_x, tm_w, args);
   return cudaGetLastError();

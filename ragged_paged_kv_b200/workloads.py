@@ -237,9 +237,12 @@ class _Req:
     gen: int = 0       # tokens generated so far
 
 
+POLICIES = ("greedy", "equal_split")
+
+
 def splitfuse_schedule(seed: int, budget: int = 2048, n_active: int = 32, n_total: int = 512,
                        prompt_mean: float = 2600.0, out_mean: float = 60.0, rel_sd: float = 0.3,
-                       events: list | None = None):
+                       events: list | None = None, policy: str = "greedy", prompts=None, outputs=None):
     """Yield (iteration, [(rid, q_len, ctx_len), ...]) for a closed loop of
     synthetic clients under a fixed token budget.
 
@@ -247,21 +250,41 @@ def splitfuse_schedule(seed: int, budget: int = 2048, n_active: int = 32, n_tota
       1. every request already generating contributes one decode token, its
          context being the prompt plus the tokens generated before it;
       2. the rest of the budget goes to requests still in their prompt, in
-         arrival order, each taking min(prompt tokens left, budget left);
+         arrival order, each taking min(prompt tokens left, share left),
+         where the share depends on ``policy``:
+           "greedy"       the whole rest of the budget (every pass is filled
+                          while prompt tokens are pending);
+           "equal_split"  the pending prompt tokens (the pool) divided evenly
+                          over the passes they need at this rest r: with
+                          n = ceil(pool / r) passes, ceil(pool / n) tokens
+                          (the card's concavity argument: throughput is
+                          concave in tokens per pass, so splitting a pool of
+                          tokens evenly across passes is optimal; "Interesting
+                          ideas" of the DeepSpeed-FastGen research-library
+                          card);
       3. a request whose prompt completes in this iteration has produced its
          first output token; a generating request produces one more;
       4. a request that has produced its G-th token leaves at the end of the
          iteration and the next arrival takes its place.
     Prompt length P = max(1, round(N(2600, 780))), output length
-    G = max(1, round(N(60, 18))).
+    G = max(1, round(N(60, 18))); ``prompts`` / ``outputs`` (sequences of
+    n_total ints) replace the draws.
     If `events` is a list, each iteration appends (iteration, produced,
     joined, left) to it after the batch has been consumed: the (rid,
     is_first_token) pairs of the tokens the iteration produced, the requests
     that became active for the next iteration and those that finished.
     """
+    if policy not in POLICIES:
+        raise ValueError(f"policy {policy!r} not in {POLICIES}")
     rng = np.random.default_rng(np.random.SeedSequence(seed, spawn_key=(_KIND_LENS,)))
     P = np.maximum(1, np.rint(rng.normal(prompt_mean, rel_sd * prompt_mean, n_total))).astype(int)
     G = np.maximum(1, np.rint(rng.normal(out_mean, rel_sd * out_mean, n_total))).astype(int)
+    if prompts is not None:
+        P = np.asarray(prompts, dtype=int)
+    if outputs is not None:
+        G = np.asarray(outputs, dtype=int)
+    if len(P) < n_total or len(G) < n_total or (P < 1).any() or (G < 1).any():
+        raise ValueError("need n_total prompt and output lengths, each >= 1")
     nxt = 0
     active: list[_Req] = []
     while len(active) < n_active and nxt < n_total:
@@ -275,11 +298,17 @@ def splitfuse_schedule(seed: int, budget: int = 2048, n_active: int = 32, n_tota
             if r.done == r.prompt and left > 0:
                 batch.append((r.rid, 1, r.prompt + r.gen - 1))
                 left -= 1
+        share = left
+        if policy == "equal_split" and left > 0:
+            pool = sum(r.prompt - r.done for r in active if r.done < r.prompt)
+            if pool > left:
+                n_pass = -(-pool // left)
+                share = -(-pool // n_pass)
         for r in active:
-            if r.done < r.prompt and left > 0:
-                c = min(r.prompt - r.done, left)
+            if r.done < r.prompt and share > 0:
+                c = min(r.prompt - r.done, share)
                 batch.append((r.rid, c, r.done))
-                left -= c
+                share -= c
         yield it, batch
         by_id = {b[0]: b for b in batch}
         still = []

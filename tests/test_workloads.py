@@ -1,6 +1,7 @@
 """Input-generator checks: determinism, the fixed-budget invariant, token
-conservation of the SplitFuse batch composer, and position-keyed generation
-(so a chunked prompt sees the same numbers as the one-shot prompt)."""
+conservation of the SplitFuse batch composer under both chunking policies,
+the equal-split policy's even passes, and position-keyed generation (so a
+chunked prompt sees the same numbers as the one-shot prompt)."""
 import numpy as np
 import pytest
 
@@ -37,10 +38,11 @@ def test_generation_is_deterministic():
         assert np.array_equal(x, y)
 
 
-def test_splitfuse_composer_conserves_tokens():
+@pytest.mark.parametrize("policy", W.POLICIES)
+def test_splitfuse_composer_conserves_tokens(policy):
     seen = {}
     for it, batch in W.splitfuse_schedule(seed=7, budget=512, n_active=8, n_total=40,
-                                          prompt_mean=900.0, out_mean=12.0):
+                                          prompt_mean=900.0, out_mean=12.0, policy=policy):
         assert sum(b[1] for b in batch) <= 512
         for rid, q, c in batch:
             seen.setdefault(rid, {}).setdefault("events", []).append((it, q, c))
@@ -89,3 +91,51 @@ def test_context_slices_are_consistent():
     k, v = w.context(1)
     k2, v2 = w.context(1, 10, 30)
     assert np.array_equal(k[10:30], k2) and np.array_equal(v[10:30], v2)
+
+
+def _passes(policy, prompts, budget, outputs=None):
+    n = len(prompts)
+    return [sum(b[1] for b in batch) for _, batch in
+            W.splitfuse_schedule(seed=0, budget=budget, n_active=n, n_total=n, policy=policy,
+                                 prompts=prompts, outputs=outputs or [1] * n)]
+
+
+def test_equal_split_spreads_one_long_prompt_evenly():
+    # 5000 prompt tokens at budget 2048 need three passes: greedy fills two
+    # and leaves 904 for the third; the even split gives 1667 + 1667 + 1666
+    assert _passes("greedy", [5000], 2048) == [2048, 2048, 904]
+    assert _passes("equal_split", [5000], 2048) == [1667, 1667, 1666]
+    # a prompt that fits is taken whole by both
+    assert _passes("equal_split", [700], 2048) == _passes("greedy", [700], 2048) == [700]
+
+
+def test_equal_split_divides_a_pool_of_prompts_evenly():
+    # pool 3000 + 1500 = 4500 tokens over three passes of 1500 (arrival order
+    # within each pass); greedy gives 2048, 2048, 404
+    assert _passes("equal_split", [3000, 1500], 2048) == [1500, 1500, 1500]
+    assert _passes("greedy", [3000, 1500], 2048) == [2048, 2048, 404]
+
+
+def test_equal_split_passes_differ_by_at_most_one_token():
+    # all requests active from the start, one output token each (no decodes):
+    # the pool only shrinks, and the passes are the even split of the pool
+    # over the fewest passes that hold it
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        n = int(rng.integers(1, 6))
+        prompts = rng.integers(1, 6000, n).tolist()
+        budget = int(rng.integers(16, 4096))
+        p = _passes("equal_split", prompts, budget)
+        total = sum(prompts)
+        assert sum(p) == total and max(p) <= budget
+        assert len(p) == -(-total // budget)
+        assert max(p) - min(p) <= 1, (prompts, budget, p)
+
+
+def test_equal_split_is_deterministic_and_never_exceeds_the_budget():
+    a = list(W.splitfuse_schedule(seed=3, budget=2048, policy="equal_split"))
+    b = list(W.splitfuse_schedule(seed=3, budget=2048, policy="equal_split"))
+    assert a == b
+    assert all(sum(x[1] for x in batch) <= 2048 for _, batch in a)
+    with pytest.raises(ValueError):
+        next(W.splitfuse_schedule(seed=3, policy="largest_first"))
