@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import (PagedCache, append_kv, attend_contiguous, bf16_bits_to_f64,
+from oracle import (PagedCache, append_kv, attend_contiguous, bf16_bits_to_f64, f64_to_bf16_bits,
                     ragged_attention, token_positions)
 from oracle.forward import splitfuse_pass
 from ragged_paged_kv_b200 import workloads as W
@@ -265,6 +265,86 @@ def test_linear_rounds_the_exact_sum_once():
         w = f32_to_bf16_bits(np.array([[1.0, 2.0 ** -8, tail]], dtype=np.float32))
         assert bf16_bits_to_f64(linear(x, w))[0, 0] == want
         assert bf16_bits_to_f64(linear(x, w ^ np.uint16(0x8000)))[0, 0] == -want
+
+
+def _tail_case(head, tail_sign):
+    """x = 4096 ones; w = two head terms, then 4094 copies of +-2^-61 (all
+    bf16 values)."""
+    x = f32_to_bf16_bits(np.ones((1, 4096), dtype=np.float32))
+    w = np.full((1, 4096), tail_sign * 2.0 ** -61, dtype=np.float32)
+    w[0, :2] = head
+    return x, f32_to_bf16_bits(w)
+
+
+def test_linear_sums_4096_terms_exactly():
+    """Two 4096-term sums that lie next to a bf16 midpoint, one on each side.
+    1 + 2^-8 + 4094 * 2^-61 is just above the midpoint of 1 and 1 + 2^-7 and
+    must round up; 1 + 3 * 2^-8 - 4094 * 2^-61 is just below the midpoint of
+    1 + 2^-7 and 1 + 2^-6 and must round down: both give 1 + 2^-7. A float64
+    sum taken left to right drops every 2^-61 term (each is under half a
+    float64 unit of the running sum), lands on the midpoint, and rounds to
+    even: the wrong word both times."""
+    from oracle import linear
+    for head, sign in (((1.0, 2.0 ** -8), 1.0), ((1.0, 3 * 2.0 ** -8), -1.0)):
+        x, w = _tail_case(head, sign)
+        assert bf16_bits_to_f64(linear(x, w))[0, 0] == 1.0 + 2.0 ** -7
+        seq = 0.0
+        for a, b in zip(bf16_bits_to_f64(x)[0], bf16_bits_to_f64(w)[0]):
+            seq += float(a) * float(b)
+        assert bf16_bits_to_f64(f64_to_bf16_bits(np.float64(seq)))[()] != 1.0 + 2.0 ** -7
+
+
+def _nearest_bf16_exact(S):
+    """Brute force on exact rationals: the bf16 word nearest the Fraction S
+    (finite, inside the bf16 range), ties to the even pattern. The candidates
+    are the three words around float(S)'s rounding."""
+    from fractions import Fraction
+    b = int(f64_to_bf16_bits(np.float64(float(S)))[()])
+    cands = []
+    for c in (b - 1, b, b + 1):
+        c &= 0xFFFF
+        v = float(bf16_bits_to_f64(np.uint16(c))[()])
+        if np.isfinite(v):
+            cands.append((abs(Fraction(v) - S), c & 1, c))
+    cands.sort()
+    best = [c for c in cands if c[0] == cands[0][0]]
+    return min(best, key=lambda c: c[1])[2] if len(best) > 1 else best[0][2]
+
+
+def test_round_exact_sum_against_rationals():
+    """round_exact_sum (the oracle's exact path) against sums of Fractions:
+    N(0,1) products, sums built to sit on a bf16 midpoint exactly (a true
+    tie) and within 2^-60 of one on either side, K from 2 to 4096."""
+    from fractions import Fraction
+    from oracle.projection import round_exact_sum
+    rng = np.random.default_rng(11)
+    cases = []
+    for K in (2, 17, 300, 4096):
+        a = bf16_bits_to_f64(f32_to_bf16_bits(rng.standard_normal(K).astype(np.float32)))
+        b = bf16_bits_to_f64(f32_to_bf16_bits(rng.standard_normal(K).astype(np.float32)))
+        cases.append(a * b)
+    for mid in (1.0 + 2.0 ** -8, -(3.0 + 2.0 ** -6), 2.0 ** -20 * (1 + 2.0 ** -8)):
+        for eps in (0.0, 2.0 ** -60, -(2.0 ** -60)):
+            t = [mid * 0.5, mid * 0.25, mid * 0.25] + [eps / 1024] * 1024 + [0.0] * 7
+            cases.append(np.array(t))
+    for terms in cases:
+        S = sum((Fraction(float(t)) for t in terms), Fraction(0))
+        assert int(round_exact_sum(terms)) == _nearest_bf16_exact(S)
+
+
+def test_linear_bound_path_agrees_with_exact_sums():
+    """The float64 path of linear (used where its error bound proves the
+    rounding) against the exact path for every output of a K = 4096 case."""
+    from oracle import linear
+    from oracle.projection import round_exact_sum
+    rng = np.random.default_rng(12)
+    x = f32_to_bf16_bits(rng.standard_normal((3, 4096)).astype(np.float32))
+    w = f32_to_bf16_bits((rng.standard_normal((24, 4096)) / 64).astype(np.float32))
+    y = linear(x, w)
+    xs, ws = bf16_bits_to_f64(x), bf16_bits_to_f64(w)
+    for t in range(3):
+        for j in range(24):
+            assert y[t, j] == round_exact_sum(xs[t] * ws[j]), (t, j)
 
 
 def test_qkv_projection_against_term_by_term_sums():

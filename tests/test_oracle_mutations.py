@@ -165,10 +165,19 @@ def _truncated(x, w):
     return (y.view(np.uint32) >> 16).astype(np.uint16)
 
 
+def _sequential_float64(x, w):
+    # an ordinary float64 sum, term after term, rounded to bf16 at the end
+    acc = np.zeros((x.shape[0], w.shape[0]))
+    for i in range(x.shape[1]):
+        acc = acc + np.outer(x[:, i], w[:, i])
+    return obf.f64_to_bf16_bits(acc)
+
+
 @pytest.mark.parametrize("mut,pin", [(_dropped_term, "test_linear_against_term_by_term_sums"),
                                      (_through_float32, "test_linear_rounds_the_exact_sum_once"),
-                                     (_truncated, "test_linear_against_term_by_term_sums")],
-                         ids=["dropped_term", "float32_sum", "truncation"])
+                                     (_truncated, "test_linear_against_term_by_term_sums"),
+                                     (_sequential_float64, "test_linear_sums_4096_terms_exactly")],
+                         ids=["dropped_term", "float32_sum", "truncation", "sequential_float64_sum"])
 def test_linear_mistakes_are_caught(monkeypatch, mut, pin):
     import oracle
     monkeypatch.setattr(oracle, "linear", _linear_with(mut))

@@ -8,7 +8,14 @@ output rounded to bf16. These tests replay it with numpy and compare against
 the exact float64 softmax (the oracle's definition), to show that the
 parity tolerances hold for the method itself:
 - max-abs 2e-2 and relative L2 5e-3 on N(0,1) data;
-- 2e-2 + 2^-8 |O| + 2^-7 A on peaked scores, with A = sum p|V| / sum p;
+- on peaked scores, the bound derived from the method's two roundings to
+  bf16 (unit roundoff 2^-8: 8 significant bits, ties to even):
+      |bf16(O_k) - O| <= 2^-8 |O| + 2^-8 (1 + 2^-8) A + e,
+  where O_k = sum bf16(p) V / sum p is the kernel's unrounded output (each
+  weight off by at most 2^-8 of itself, so O_k is within 2^-8 A of O, with
+  A = sum p|V| / sum p), the output rounding adds at most 2^-8 |O_k|, and e
+  collects the fp32 effects (scores, ex2.approx, sums), covered by the fixed
+  2e-2;
 - splitting and combining moves the result by no more than the bf16
   rounding of P does: each piece rounds its weights against its own running
   maximum, so the rounding errors differ, bounded by 2^-8 A.
@@ -59,6 +66,12 @@ def combine(parts):
     return O / L[:, None]
 
 
+def peaked_bound(ref, mass):
+    """The derived per-output bound (module docstring), with the fixed 2e-2
+    standing for the fp32 effects."""
+    return 2e-2 + 2.0 ** -8 * np.abs(ref) + 2.0 ** -8 * (1 + 2.0 ** -8) * mass
+
+
 def case(rng, rows, keys, d, q_scale):
     q = bf16(rng.standard_normal((rows, d)) * q_scale)
     K = bf16(rng.standard_normal((keys, d)))
@@ -85,7 +98,7 @@ def test_peaked_scores_meet_the_derived_bound():
         ref, mass = exact(q, K, V, scale)
         O, m, l = online(q, K, V, scale)
         got = bf16(O / l[:, None])
-        bound = 2e-2 + 2.0 ** -8 * np.abs(ref) + 2.0 ** -7 * mass
+        bound = peaked_bound(ref, mass)
         assert np.all(np.abs(got - ref) <= bound)
         assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 5e-3
         # the rescale really ran: the running maximum moved after the first tile
@@ -104,3 +117,43 @@ def test_split_and_combine_stays_within_the_weight_rounding():
             parts = [online(q, K[:cut], V[:cut], scale), online(q, K[cut:], V[cut:], scale)]
             both = combine(parts)
             assert np.all(np.abs(both - one) <= 2.0 ** -8 * mass + 1e-6)
+
+
+def test_replay_of_the_peaked_grouped_query_case():
+    """The GPU parity case with peaked scores at 8/2 heads, d = 64 (queries
+    times 16): its 300-token prompt chunk at context 0 runs on the query-tile
+    kernel, the method replayed here. On the same data (the oracle's rotated
+    queries and cache, every chunk row and head) the method itself exceeds
+    the fixed 2e-2 on an output above 4 in magnitude, where rounding to bf16
+    alone can move a value by 2^-6, and every output stays within the derived
+    bound: an error of that size is the method's, not a kernel defect."""
+    from oracle import PagedCache
+    from oracle.forward import splitfuse_pass
+    from ragged_paged_kv_b200 import fixtures
+    from ragged_paged_kv_b200 import workloads as W
+    w = W._make("peaked_gqa_d64", 8, 2, 64, 16, [0, 1, 2, 3], [300, 1, 1, 17], [0, 3000, 700, 500],
+                seed=41, budget=319)
+    q0, k, v = w.qkv()
+    q = f64_to_bf16_bits(bf16_bits_to_f64(q0) * 16.0)
+    pc = PagedCache(w.n_blocks, w.n_kv_heads, w.block_size, w.head_dim, fill=fixtures.SENTINEL)
+    for s_ in range(w.n_seqs):
+        ids, blocks = fixtures.context_blocks(w, s_)
+        for i, b in enumerate(ids):
+            pc.blocks[int(b)] = blocks[i].copy()
+    q_rot, _, ref = splitfuse_pass(pc, w.block_tables, w.q_lens, w.ctx_lens, q, k, v, w.rope_theta,
+                                   w.softmax_scale, 0)
+    K, V = (bf16_bits_to_f64(a) for a in pc.gather(w.block_tables[0], int(w.q_lens[0])))
+    g = w.n_q_heads // w.n_kv_heads
+    errs, over = [], 0
+    for t in range(int(w.q_lens[0])):
+        for h in range(w.n_q_heads):
+            qv = bf16_bits_to_f64(q_rot[t, h])[None, :]
+            Kh, Vh = K[:t + 1, h // g], V[:t + 1, h // g]
+            O, m, l = online(qv, Kh, Vh, w.softmax_scale)
+            got = bf16(O / l[:, None])[0]
+            _, mass = exact(qv, Kh, Vh, w.softmax_scale)
+            err = np.abs(got - ref[t, h])
+            assert np.all(err <= peaked_bound(ref[t, h], mass[0])), (t, h)
+            over += int(np.sum((err > 2e-2) & (np.abs(ref[t, h]) > 4)))
+            errs.append(err.max())
+    assert over >= 1 and max(errs) > 2e-2
