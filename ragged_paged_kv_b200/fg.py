@@ -11,7 +11,10 @@ import re
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libfg.so")
+# RAGGED_PAGED_KV_LIB=trace selects the instrumented build (libfg_trace.so:
+# the same kernels plus cycle accounting in the query-tile kernel)
+LIB_PATH = os.path.join(_PKG, "libfg_trace.so" if os.environ.get("RAGGED_PAGED_KV_LIB") == "trace"
+                        else "libfg.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fg.h")
 
 STATUS = {0: "FG_OK", 1: "FG_ERR_INVALID_ARG", 2: "FG_ERR_OUT_OF_RANGE", 3: "FG_ERR_ALIAS",
@@ -74,6 +77,9 @@ def lib() -> ctypes.CDLL:
     L.fg_status_string.restype = ctypes.c_char_p
     L.fg_last_error.argtypes = []
     L.fg_last_error.restype = ctypes.c_char_p
+    if hasattr(L, "fg_phase_trace_read"):  # the trace build only
+        L.fg_phase_trace_read.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int, ctypes.c_int]
+        L.fg_phase_trace_read.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -365,3 +371,81 @@ def forward_host(cache: KVCache, batch: RaggedBatch, host_in: dict, dev: dict, h
         forward(cache, batch, dev["q"], dev["k"], dev["v"], dev["q_rot"], dev["out"], n_q_heads,
                 rope_theta, softmax_scale, sliding_window, s)
         host_out.copy_(dev["out"], non_blocking=True)
+
+
+class HostPipeline:
+    """Passes from pinned host memory with the copies overlapped across passes.
+
+    Each pass copies its q, k, v from pinned host memory to the device, runs
+    rotary + append and the ragged attention (fg_rotary_kv_append,
+    fg_ragged_attention), and copies the output back to pinned host memory.
+    The host-to-device copy of pass i + 1 runs on an upload stream and the
+    device-to-host copy of pass i - 1 on a download stream while pass i
+    computes on the compute stream (PCIe carries both directions at once);
+    two device buffer sets are used in turn, and events order each copy
+    after the pass that last used its buffers. submit() only enqueues; a
+    pass's host buffers must stay untouched until wait() for it returns.
+    The batch metadata of each pass is put on the compute stream, so one
+    batch handle serves every pass (its uploads are double-buffered)."""
+
+    def __init__(self, cache: "KVCache", max_tokens: int, n_q_heads: int, device=None):
+        import torch
+        dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        d, hkv = cache.head_dim, cache.n_kv_heads
+        mk = lambda h: torch.empty((max_tokens, h, d), dtype=torch.bfloat16, device=dev)
+        self.cache, self.n_q_heads, self.max_tokens = cache, int(n_q_heads), int(max_tokens)
+        self.bufs = [{"q": mk(n_q_heads), "k": mk(hkv), "v": mk(hkv), "q_rot": mk(n_q_heads),
+                      "out": mk(n_q_heads)} for _ in range(2)]
+        self.up, self.comp, self.down = (torch.cuda.Stream(device=dev) for _ in range(3))
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]
+        # inputs uploaded; inputs consumed (append done); output ready; output downloaded
+        self.ev_up, self.ev_in_free, self.ev_done, self.ev_out_free = ev(), ev(), ev(), ev()
+        self.n = 0
+
+    def submit(self, batch: "RaggedBatch", seq_ids, q_lens, ctx_lens, block_tables, host_q, host_k,
+               host_v, host_out, rope_theta: float, softmax_scale: float, sliding_window: int = 0) -> int:
+        """Enqueue one pass; returns its index (for wait())."""
+        import torch
+        T = int(np.asarray(q_lens, dtype=np.int64).sum())
+        if T > self.max_tokens:
+            raise ValueError(f"{T} tokens > max_tokens {self.max_tokens}")
+        for name, t in (("host_q", host_q), ("host_k", host_k), ("host_v", host_v), ("host_out", host_out)):
+            if t.is_cuda or not t.is_pinned() or t.shape[0] != T:
+                raise ValueError(f"{name} must be pinned host memory with {T} rows")
+        j = self.n % 2
+        b = self.bufs[j]
+        if self.n >= 2:
+            self.up.wait_event(self.ev_in_free[j])
+        with torch.cuda.stream(self.up):
+            b["q"][:T].copy_(host_q, non_blocking=True)
+            b["k"][:T].copy_(host_k, non_blocking=True)
+            b["v"][:T].copy_(host_v, non_blocking=True)
+            self.ev_up[j].record(self.up)
+        self.comp.wait_event(self.ev_up[j])
+        if self.n >= 2:
+            self.comp.wait_event(self.ev_out_free[j])
+        batch.put(self.cache, seq_ids, q_lens, ctx_lens, block_tables, self.comp)
+        rotary_kv_append(self.cache, batch, b["q"][:T], b["k"][:T], b["v"][:T], b["q_rot"][:T],
+                         self.n_q_heads, rope_theta, self.comp)
+        self.ev_in_free[j].record(self.comp)
+        ragged_attention(self.cache, batch, b["q_rot"][:T], b["out"][:T], self.n_q_heads, softmax_scale,
+                         sliding_window, self.comp)
+        self.ev_done[j].record(self.comp)
+        self.down.wait_event(self.ev_done[j])
+        with torch.cuda.stream(self.down):
+            host_out.copy_(b["out"][:T], non_blocking=True)
+            self.ev_out_free[j].record(self.down)
+        self.n += 1
+        return self.n - 1
+
+    def wait(self, i: int):
+        """Block until pass i's output is in host memory (the last two
+        passes can be waited for)."""
+        if not (self.n - 2 <= i < self.n):
+            raise ValueError(f"pass {i} is not one of the last two of {self.n}")
+        self.ev_out_free[i % 2].synchronize()
+
+    def drain(self):
+        self.down.synchronize()
+        self.comp.synchronize()
+        self.up.synchronize()

@@ -299,6 +299,44 @@ def test_append_without_rotary(which):
     _free(cache, batch)
 
 
+def pair_mag(pre_bits):
+    """|x_i| + |x_{i+d/2}| for bf16 vectors [..., d]: a rotated value moves by
+    at most about a bf16 unit of this when its inputs are off by one unit
+    each."""
+    x = np.abs(bf16_to_f64(pre_bits))
+    h = x.shape[-1] // 2
+    m = x[..., :h] + x[..., h:]
+    return np.concatenate([m, m], axis=-1)
+
+
+def fp32_sum_error(x_bits, w_bits):
+    """Per output of x W^T: the bound gamma_K * sum_i |x_i w_i| on how far an
+    fp32 sum of the K exact products (in any order) can be from the exact sum,
+    gamma_K = K 2^-24. Where the terms cancel, this exceeds a bf16 unit of the
+    result itself."""
+    K = x_bits.shape[1]
+    return K * 2.0 ** -24 * (np.abs(bf16_to_f64(x_bits)) @ np.abs(bf16_to_f64(w_bits)).T)
+
+
+def pair_sum(a):
+    """a_i + a_{i+d/2} for [..., d] arrays, repeated over both halves: how a
+    per-input bound carries through the rotation (|cos|, |sin| <= 1)."""
+    h = a.shape[-1] // 2
+    m = a[..., :h] + a[..., h:]
+    return np.concatenate([m, m], axis=-1)
+
+
+def near(got_bits, ref_bits, scale, what, acc=0.0):
+    """Every word within two bf16 units (of scale + |ref|) plus `acc`, the
+    fp32 accumulation bound of its inputs, and under 1 % of the words
+    different: the bar for values computed from projected inputs, whose fp32
+    sums may round to the neighbouring bf16 of the exact sum's rounding."""
+    g, r = bf16_to_f64(got_bits), bf16_to_f64(ref_bits)
+    excess = np.abs(g - r) - (2.0 ** -6 * (scale + np.abs(r)) + acc)
+    assert np.all(excess <= 0), f"{what}: beyond two bf16 units plus the fp32 sum bound by {excess.max():.3g}"
+    assert np.mean(got_bits != ref_bits) < 0.01, f"{what}: {np.mean(got_bits != ref_bits):.3%} words differ"
+
+
 @pytest.mark.parametrize("which", ["mha_d64", "gqa_d128"])
 def test_fused_qkv_projection_rotary_append(which):
     """fg_qkv_rotary_kv_append: the projection x W^T fused with rotary and the
@@ -340,20 +378,12 @@ def test_fused_qkv_projection_rotary_append(which):
     q_ref, k_ref, ref = splitfuse_pass(pc, w.block_tables, w.q_lens, w.ctx_lens, q, k, v, w.rope_theta,
                                        w.softmax_scale, w.sliding_window)
 
-    def pair_mag(pre_bits):
-        # |x_i| + |x_{i+d/2}|: a rotated value moves by at most about a bf16
-        # unit of this when its inputs are off by one unit each
-        x = np.abs(bf16_to_f64(pre_bits))
-        h = x.shape[-1] // 2
-        m = x[..., :h] + x[..., h:]
-        return np.concatenate([m, m], axis=-1)
-
-    def near(got_bits, ref_bits, scale, what):
-        g, r = bf16_to_f64(got_bits), bf16_to_f64(ref_bits)
-        assert np.all(np.abs(g - r) <= 2.0 ** -6 * (scale + np.abs(r))), f"{what}: beyond two bf16 units"
-        assert np.mean(got_bits != ref_bits) < 0.01, f"{what}: {np.mean(got_bits != ref_bits):.3%} words differ"
-
-    near(to_bits(q_rot), q_ref, pair_mag(q), "q_rot")
+    acc = fp32_sum_error(x_bits, w_bits)
+    hq, hkv, d = w.n_q_heads, w.n_kv_heads, w.head_dim
+    acc_q = pair_sum(acc[:, :hq * d].reshape(-1, hq, d))
+    acc_k = pair_sum(acc[:, hq * d:(hq + hkv) * d].reshape(-1, hkv, d))
+    acc_v = acc[:, (hq + hkv) * d:].reshape(-1, hkv, d)
+    near(to_bits(q_rot), q_ref, pair_mag(q), "q_rot", acc_q)
     cu = np.concatenate([[0], np.cumsum(w.q_lens)])
     for s in range(w.n_seqs):
         ids = w.block_tables[s, :w.blocks_used(s)].astype(np.int64)
@@ -368,9 +398,107 @@ def test_fused_qkv_projection_rotary_append(which):
                 new_v.append(dev[bi, 1, :, sl])
             else:  # prior context and slots past the end: untouched, bit for bit
                 assert np.array_equal(dev[bi, :, :, sl], ref_blocks[bi, :, :, sl]), f"slot {pos} of seq {s}"
-        near(np.stack(new_k), k_ref[tok], pair_mag(k[tok]), f"new K of seq {s}")
-        near(np.stack(new_v), v[tok], 0.0, f"new V of seq {s}")
+        near(np.stack(new_k), k_ref[tok], pair_mag(k[tok]), f"new K of seq {s}", acc_k[tok])
+        near(np.stack(new_v), v[tok], 0.0, f"new V of seq {s}", acc_v[tok])
     assert_close(bf16_to_f64(to_bits(out)), ref, w.name)
+    _free(cache, batch)
+
+
+def test_host_pipeline_matches_device_passes():
+    """fg.HostPipeline: four passes of a small grouped-query batch from pinned
+    host buffers, each with its own q, k, v, enqueued back to back (uploads,
+    computes and downloads of neighbouring passes overlap). Each output, read
+    after wait(), equals the same four passes run one after the other on
+    device tensors on an identical cache, bit for bit."""
+    w = W._make("pipe_gqa", 8, 2, 128, 64, [0, 1, 2], [70, 1, 1], [100, 3000, 200], seed=13, budget=72)
+    T = w.n_tokens
+    caches = []
+    for _ in range(2):
+        c = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+        fixtures.fill(c.tensor)
+        fixtures.write_context(w, c.tensor)
+        caches.append(c)
+    g = torch.Generator().manual_seed(5)
+    passes = [tuple(torch.randn((T, h, w.head_dim), generator=g).to(torch.bfloat16)
+                    for h in (w.n_q_heads, w.n_kv_heads, w.n_kv_heads)) for _ in range(4)]
+    # reference: device tensors, one pass after the other
+    b_ref = fg.RaggedBatch(T, w.n_seqs, w.block_tables.shape[1])
+    refs = []
+    for q, k, v in passes:
+        b_ref.put(caches[0], w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables)
+        qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+        q_rot, out = torch.empty_like(qd), torch.empty_like(qd)
+        fg.forward(caches[0], b_ref, qd, kd, vd, q_rot, out, w.n_q_heads, w.rope_theta, w.softmax_scale)
+        torch.cuda.synchronize()
+        refs.append(to_bits(out))
+    # pipelined from pinned host buffers
+    b = fg.RaggedBatch(T, w.n_seqs, w.block_tables.shape[1])
+    pipe = fg.HostPipeline(caches[1], T, w.n_q_heads)
+    host = [(q.pin_memory(), k.pin_memory(), v.pin_memory(), torch.empty_like(q).pin_memory())
+            for q, k, v in passes]
+    for i, (q, k, v, o) in enumerate(host):
+        assert pipe.submit(b, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, q, k, v, o,
+                           w.rope_theta, w.softmax_scale) == i
+    pipe.wait(3)
+    pipe.drain()
+    b.device_status()
+    for i, (_, _, _, o) in enumerate(host):
+        assert np.array_equal(o.view(torch.int16).numpy().view(np.uint16), refs[i]), f"pass {i} differs"
+    _free(*caches, b, b_ref)
+
+
+def test_fused_qkv_projection_at_llama7b_width():
+    """fg_qkv_rotary_kv_append in the configuration the bench times: the
+    headline batch's 2048 tokens (31 decodes + a 2017-token chunk) at hidden
+    4096, 96 heads of 128 outputs (16 token tiles x 96 heads = 1536 CTAs, 64
+    K-slices of 64 through the ring). The oracle projects sampled token rows
+    exactly (tile edges, the decodes, the last rows, random rows), rotates
+    them at their positions, and the GPU's rotated q and the new K and V cache
+    slots of those tokens must be within two bf16 units plus the fp32
+    accumulation bound of a 4096-term sum (which dominates where the terms
+    cancel) with under 1 % of the words different."""
+    from oracle import qkv_projection
+    from oracle.rotary import rotate_half
+    w = W.config2()
+    hidden, T = 4096, w.n_tokens
+    rng = np.random.default_rng(41)
+    x_bits = W.f32_to_bf16_bits(rng.standard_normal((T, hidden), dtype=np.float32))
+    n_out = (w.n_q_heads + 2 * w.n_kv_heads) * w.head_dim
+    w_bits = W.f32_to_bf16_bits(rng.standard_normal((n_out, hidden), dtype=np.float32) / np.float32(64.0))
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+    fixtures.fill(cache.tensor)
+    batch = fg.RaggedBatch(T, w.n_seqs, w.block_tables.shape[1])
+    batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables)
+    xd = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    wd = torch.from_numpy(w_bits.view(np.int16)).cuda().view(torch.bfloat16)
+    q_rot = torch.full((T, w.n_q_heads, w.head_dim), float("nan"), dtype=torch.bfloat16, device="cuda")
+    fg.qkv_rotary_kv_append(cache, batch, xd, wd, q_rot, w.n_q_heads, w.rope_theta)
+    torch.cuda.synchronize()
+    batch.device_status()
+    cu = w.cu_q
+    tok_seq = np.repeat(np.arange(w.n_seqs), w.q_lens)
+    pos = np.concatenate([np.arange(c, c + q) for q, c in zip(w.q_lens, w.ctx_lens)])
+    rows = {0, 1, 126, 127, 128, 129, 1023, 1024, 1025, T - 2, T - 1}
+    rows |= {int(cu[s]) for s in range(w.n_seqs) if w.q_lens[s] == 1}
+    rows |= set(rng.choice(T, 16, replace=False).tolist())
+    rows = np.array(sorted(rows), dtype=np.int64)
+    q, k, v = qkv_projection(x_bits[rows], w_bits, w.n_q_heads, w.n_kv_heads, w.head_dim)
+    q_ref = rotate_half(q, pos[rows], w.rope_theta)
+    k_ref = rotate_half(k, pos[rows], w.rope_theta)
+    hq, hkv, d = w.n_q_heads, w.n_kv_heads, w.head_dim
+    acc = fp32_sum_error(x_bits[rows], w_bits)
+    acc_q = pair_sum(acc[:, :hq * d].reshape(-1, hq, d))
+    acc_k = pair_sum(acc[:, hq * d:(hq + hkv) * d].reshape(-1, hkv, d))
+    acc_v = acc[:, (hq + hkv) * d:].reshape(-1, hkv, d)
+    near(to_bits(q_rot)[rows], q_ref, pair_mag(q), "q_rot", acc_q)
+    blk = np.array([w.block_tables[tok_seq[r], pos[r] // w.block_size] for r in rows], dtype=np.int64)
+    slot = torch.from_numpy(pos[rows] % w.block_size).cuda()
+    dev = cache.tensor[torch.from_numpy(blk).cuda()]            # [n, 2, Hkv, B, d]
+    ar = torch.arange(len(rows), device="cuda")
+    k_dev = to_bits(dev[ar, 0, :, slot])                          # [n, Hkv, d]
+    v_dev = to_bits(dev[ar, 1, :, slot])
+    near(k_dev, k_ref, pair_mag(k), "new K slots", acc_k)
+    near(v_dev, v, 0.0, "new V slots", acc_v)
     _free(cache, batch)
 
 
@@ -444,13 +572,18 @@ def test_peaked_scores_exercise_the_running_max_rescale(which):
 
     With the softmax this peaked an output is close to one V row, so outputs
     reach |V| ~ 5, where the fixed 2e-2 bound of the O(1) cases no longer
-    covers bf16 itself: rounding the exact result to bf16 alone moves it by
-    up to 2^-8 |O| (0.0156 at |O| in [4, 8)). The weights P enter the P.V
-    product rounded to bf16 (relative 2^-9 each) while their sum is kept in
-    fp32, which moves O by at most 2^-9 A, A = sum p |V| / sum p (the same
-    attention over |V|, computed by the oracle). Each output is therefore
-    held to 2e-2 + 2^-8 |O| + 2^-7 A (four times the weight term), and the
-    relative L2 error to the usual 5e-3."""
+    covers bf16 itself: bf16 keeps 8 significant bits (unit roundoff 2^-8),
+    so rounding the output alone moves it by up to 2^-8 |O| (0.0156 at |O|
+    in [4, 8)). The weights P enter the P.V product rounded to bf16 (each
+    off by at most 2^-8 of itself) while their sum is kept in fp32, which
+    moves the unrounded output by at most 2^-8 A, A = sum p |V| / sum p (the
+    same attention over |V|, computed by the oracle), and the output rounding
+    then acts on that moved value. Each output is therefore held to
+    2e-2 + 2^-8 |O| + 2^-8 (1 + 2^-8) A, the 2e-2 standing for the fp32
+    effects (scores, ex2.approx, sums), and the relative L2 error to the
+    usual 5e-3. The host replay of the kernels' method on the d = 64
+    grouped-query case (tests/test_softmax_method.py) shows the method
+    itself passing 2e-2 on an output above 4."""
     from oracle.bf16 import f64_to_bf16_bits
     shapes = {"mha_d128": (32, 32, 128, 64), "gqa_d64": (8, 2, 64, 16), "mha_d64": (4, 4, 64, 16)}
     Hq, Hkv, d, B = shapes[which]
@@ -489,7 +622,7 @@ def test_peaked_scores_exercise_the_running_max_rescale(which):
     got = bf16_to_f64(to_bits(out))
     assert np.isfinite(got).all()
     err = np.abs(got - ref)
-    bound = MAX_ABS + 2.0 ** -8 * np.abs(ref) + 2.0 ** -7 * mass
+    bound = MAX_ABS + 2.0 ** -8 * np.abs(ref) + 2.0 ** -8 * (1 + 2.0 ** -8) * mass
     assert np.all(err <= bound), f"{w.name}: max excess {np.max(err - bound):.3g}"
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert rel <= REL_L2, f"{w.name}: rel-L2 {rel:.3g}"
