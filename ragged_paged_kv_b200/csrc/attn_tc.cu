@@ -14,9 +14,10 @@
 //   warp 8, lane 0    Q of both query tiles once per unit (3-D boxes: 64
 //                     dims x g heads x 128/g tokens), then K tiles through the
 //                     block table into a 5-stage ring;
-//   warp 8, lane 1    V tiles, the same way, into a 4-stage ring (separate
+//   warp 11, lane 0   V tiles, the same way, into a 4-stage ring (separate
 //                     streams, so a K load never waits behind a V stage that
-//                     an earlier P.V still occupies);
+//                     an earlier P.V still occupies, and separate warps, so
+//                     neither loader's loop is serialised behind the other's);
 //   warps 9, 10 (MMA) one thread per query tile issues S_t = Q_t K^T into
 //                     double-buffered TMEM S tiles and O_t += P_t V into its
 //                     TMEM O tile, with P read from tensor memory; the two
@@ -51,6 +52,50 @@ namespace {
 
 constexpr long long kWaitLimit = 1LL << 31;
 
+// Cycle accounting of the kernel's roles, compiled in only with
+// -DFG_PHASE_TRACE (the separate trace build, libfg_trace.so). Each role keeps
+// one clock64 stamp and, at every mark, adds the cycles since the previous
+// mark to one of its slots; one recording thread per role adds its slots to
+// g_phase at exit, which fg_phase_trace_read returns. Slot layout: softmax
+// of query tile t at 12 t (wait S, load S, max, rescale O, exponentials and
+// P store, V zeroing, store wait and P arrive, epilogue wait, epilogue
+// stores, unit pop, 64-key steps, wait for the exponential turn), MMA thread t at 24 + 8 t (unit
+// pop, wait K, issue S, wait V, wait P, wait O free, issue P.V, steps), the
+// K and V loaders at 40 and 48 (unit pop, wait Q free, wait stage free,
+// issue, tiles), CTA cycles and CTAs at 56 and 57; %globaltimer (ns) of the
+// first CTA start, the last CTA start and the last CTA end at 58, 59, 60
+// (minimum / maximum over the launches since the last read).
+#ifdef FG_PHASE_TRACE
+constexpr int kPhaseSlots = 64;
+__device__ unsigned long long g_phase[kPhaseSlots];
+#define PH_DECL        \
+  uint32_t ph_[12] = {}; \
+  uint32_t ph_t_ = (uint32_t)clock()
+#define PH_MARK(i)                          \
+  do {                                      \
+    const uint32_t t_ = (uint32_t)clock();  \
+    ph_[i] += t_ - ph_t_;                   \
+    ph_t_ = t_;                             \
+  } while (0)
+#define PH_COUNT(i, n) (ph_[i] += (n))
+#define PH_FLUSH(rec, base, n)                                                     \
+  do {                                                                             \
+    if (rec)                                                                       \
+      for (int i_ = 0; i_ < (n); ++i_) atomicAdd(&g_phase[(base) + i_], (unsigned long long)ph_[i_]); \
+  } while (0)
+#else
+#define PH_DECL
+#define PH_MARK(i) \
+  do {             \
+  } while (0)
+#define PH_COUNT(i, n) \
+  do {                 \
+  } while (0)
+#define PH_FLUSH(rec, base, n) \
+  do {                         \
+  } while (0)
+#endif
+
 template <int D>
 struct TcCfg {
   static constexpr int BM = 128;  // query rows per tile
@@ -65,10 +110,11 @@ struct TcCfg {
   static constexpr int kOffV = kOffK + KST * kKVBytes;
   static constexpr int kOffBar = kOffV + VST * kKVBytes;
   // q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST],
-  // then per query tile: s_full[2], p_full[2], pv_done[2], o_free; unit queue
-  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + NQ * 7 + 2 * UnitQueue::kDepth;
+  // then per query tile: s_full[2], p_full[2], pv_done[2], o_free; the
+  // exponential turns of the 4 softmax warp pairs (turn[2 r + t]); unit queue
+  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + NQ * 7 + 8 + 2 * UnitQueue::kDepth;
   static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + UnitQueue::kDepth * 4;
-  static constexpr int kThreads = 352;  // 8 softmax warps, the load warp, one MMA warp per query tile
+  static constexpr int kThreads = 384;  // 8 softmax warps, the K loader, two MMA warps, the V loader
   static constexpr uint32_t kTmemCols = 512;
   // query tile t: S (then P) buffers at kColS0 + 2 t BN and + BN, O at kColO0 + t D
   static constexpr uint32_t kColS0 = 0;
@@ -123,6 +169,44 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x for a pair of floats on the FMA pipe, without the special-function
+// unit: Cody-Waite range reduction x = j + f, j = rint(x), |f| <= 1/2, and
+// 2^x = 2^j p(f), p the degree-5 polynomial of least maximum relative error
+// to 2^f on [-1/2, 1/2] (float32 coefficients from exp2_poly_fit.py; relative
+// error 2^-22.6 before the float32 evaluation). rint(x) is an add of
+// 1.5 * 2^23, after which the low mantissa bits of the sum hold j; 2^j is
+// placed by adding (sum bits) << 23 to p's bits (the constant's own low bits
+// are zero, so only j << 23 remains). x is clamped at -127, so j >= -127
+// with f >= 0 there and the result stays a non-negative float (a subnormal
+// at the bottom); -inf, the masked keys, gives a value below 2^-148 that
+// rounds to bf16 zero.
+constexpr float kExp2C0 = 0x1.000002p+0f, kExp2C1 = 0x1.62e428p-1f, kExp2C2 = 0x1.ebf918p-3f,
+                kExp2C3 = 0x1.c6b6e4p-5f, kExp2C4 = 0x1.3d0c52p-7f, kExp2C5 = 0x1.5c08e6p-10f;
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 j = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(kExp2C5, kExp2C5), f, make_float2(kExp2C4, kExp2C4));
+  p = __ffma2_rn(p, f, make_float2(kExp2C3, kExp2C3));
+  p = __ffma2_rn(p, f, make_float2(kExp2C2, kExp2C2));
+  p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
+  p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+// Every kExp2FmaEvery-th pair of a row's exponentials goes to ex2_fma2, the
+// rest to ex2 (0: none, the default). Measured on B200 on the long-prompt
+// batch, taking a quarter or half of the exponentials off the
+// special-function unit this way made the kernel slower (the softmax's
+// instruction count, not the special-function unit, set its pace), so it is
+// off; the path stays compiled in with -DFG_EXP2_FMA_EVERY=n.
+#ifndef FG_EXP2_FMA_EVERY
+#define FG_EXP2_FMA_EVERY 0
+#endif
+constexpr int kExp2FmaEvery = FG_EXP2_FMA_EVERY;
+
 // 3-input maximum (sm_100): one instruction for two comparisons.
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float m;
@@ -150,7 +234,7 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int
 }
 
 template <int D>
-__global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+__global__ void __launch_bounds__(384, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                         const __grid_constant__ CUtensorMap tm_kv,
                                                         TcArgs a) {
   using C = TcCfg<D>;
@@ -158,6 +242,14 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
   unsigned char* smem = smem_raw;
   // SMs outside the kernel's share are left to the decode kernel
   if (ptx::sm_id() >= a.sm_end) return;
+#ifdef FG_PHASE_TRACE
+  const long long cta_t0 = clock64();
+  if (threadIdx.x == 0) {
+    const unsigned long long g0 = ptx::global_timer_ns();
+    atomicMin(&g_phase[58], g0);
+    atomicMax(&g_phase[59], g0);
+  }
+#endif
   // the swizzled tiles need 1024-byte alignment of the dynamic window
   if (ptx::smem_u32(smem_raw) & 1023u) {
     if (threadIdx.x == 0) atomicOr(a.batch.err, kErrBadIndex);
@@ -178,7 +270,12 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
   auto p_full = [tb](int t, int b) { return tb + 7 * t + 2 + b; };
   auto pv_done = [tb](int t, int b) { return tb + 7 * t + 4 + b; };
   auto o_free = [tb](int t) { return tb + 7 * t + 6; };
-  uint64_t* uq_full = tb + 7 * C::NQ;
+  // warp r of query tile 0 and warp r of tile 1 (warps r and r + 4) share an
+  // SM sub-partition and its special-function unit: they take turns with
+  // their exponentials, tile 0 first in each K/V tile; turn[2 r + t] is
+  // completed when it is tile t's turn
+  uint64_t* turn = tb + 7 * C::NQ;
+  uint64_t* uq_full = turn + 8;
   uint64_t* uq_empty = uq_full + UnitQueue::kDepth;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   // units come from a global counter through this queue (the V loader, the
@@ -209,6 +306,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       }
       ptx::mbar_init(o_free(t), 4);
     }
+    for (int i = 0; i < 8; ++i) ptx::mbar_init(&turn[i], 1);
     uq.init();
     ptx::fence_mbar_init();
   }
@@ -222,10 +320,10 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
-  if (warp == 8) {
+  if (warp == 8 || warp == 11) {
     // ---------------------------------------------------------------- loads
-    if (lane < 2) {
-      const bool is_k = lane == 0;
+    if (lane == 0) {
+      const bool is_k = warp == 8;
       const int B = a.cache.block_size;
       const int BR = B < 64 ? B : 64;
       const int Hkv = a.cache.n_kv_heads;
@@ -235,6 +333,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       uint64_t* empty = is_k ? k_empty : v_empty;
       unsigned char* ring = is_k ? sK : sV;
       int gt = 0, un = 0;
+      PH_DECL;
       for (;; ++un) {
         int u = -1;
         const bool got = is_k ? uq.push_next(un, a.counter, a.n_items, kWaitLimit, &u)
@@ -245,10 +344,12 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         }
         if (u < 0 || !ok) break;
         const Unit x = load_unit(a, u, C::BN);
+        PH_MARK(0);
         if (is_k) {
           // both query tiles' boxes (tile 1's reaches past the unit's rows
           // when R <= 128; those rows are never used)
           if (un >= 1 && !wait_or_flag(q_empty, (un - 1) & 1, err, ok)) break;
+          PH_MARK(1);
           ptx::mbar_arrive_expect_tx(q_full, C::NQ * C::kQBytes);
 #pragma unroll
           for (int t = 0; t < C::NQ; ++t)
@@ -259,32 +360,53 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         }
         const int32_t* bt = a.batch.bt + a.batch.bt_off[x.s];
         const int nb = a.batch.bt_off[x.s + 1] - a.batch.bt_off[x.s];
+        // block ids of a tile's 64 / BR boxes (-1: past the table, no load);
+        // the next tile's are read before this tile waits for its stage, so
+        // the dependent global read is off the issue path
+        constexpr int kMaxBoxes = 4;  // 64-key tile over 16-slot blocks
+        auto tile_blocks = [&](int i, int32_t (&ids)[kMaxBoxes]) {
+#pragma unroll
+          for (int j = 0; j < kMaxBoxes; ++j) {
+            const int pos = x.k00 + i * C::BN + j * BR;
+            const int lb = pos / B;
+            ids[j] = (j * BR < C::BN && lb < nb) ? bt[lb] : -1;
+          }
+        };
+        int32_t cur[kMaxBoxes], nxt[kMaxBoxes];
+        if (x.n_tiles > 0) tile_blocks(0, cur);
         for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
+          if (i + 1 < x.n_tiles) tile_blocks(i + 1, nxt);
           const int k0 = x.k00 + i * C::BN;
           uint32_t bytes = 0;
-          for (int pos = k0; pos < k0 + C::BN; pos += BR) {
-            const int lb = pos / B;
-            if (lb < nb && bt[lb] >= 0 && bt[lb] < a.cache.n_blocks) bytes += BR * 128 * C::DH;
-          }
+#pragma unroll
+          for (int j = 0; j < kMaxBoxes; ++j)
+            if (cur[j] >= 0 && cur[j] < a.cache.n_blocks) bytes += BR * 128 * C::DH;
           const int st = gt % NST;
           if (gt >= NST && !wait_or_flag(&empty[st], ((gt / NST) - 1) & 1, err, ok)) break;
+          PH_MARK(2);
+          PH_COUNT(4, 1);
           ptx::mbar_arrive_expect_tx(&full[st], bytes);
-          for (int pos = k0; pos < k0 + C::BN; pos += BR) {
-            const int lb = pos / B;
-            if (lb >= nb) continue;
-            const int32_t blk = bt[lb];
+#pragma unroll
+          for (int j = 0; j < kMaxBoxes; ++j) {
+            const int pos = k0 + j * BR;
+            const int32_t blk = cur[j];
+            if (j * BR >= C::BN || (blk == -1 && pos / B >= nb)) continue;
             if (blk < 0 || blk >= a.cache.n_blocks) {
               if (is_k) atomicOr(err, kErrBadBlock);
               continue;
             }
-            const int row = (int)((((int64_t)blk * 2 + kv) * Hkv + x.h) * B + (pos - lb * B));
+            const int row = (int)((((int64_t)blk * 2 + kv) * Hkv + x.h) * B + (pos - (pos / B) * B));
 #pragma unroll
             for (int dh = 0; dh < C::DH; ++dh)
               ptx::tma_load_2d(ring + st * C::kKVBytes + dh * C::BN * 128 + (pos - k0) * 128, &tm_kv, dh * 64,
                                row, &full[st]);
           }
+#pragma unroll
+          for (int j = 0; j < kMaxBoxes; ++j) cur[j] = nxt[j];
+          PH_MARK(3);
         }
       }
+      PH_FLUSH(true, is_k ? 40 : 48, 5);
       // every unit is claimed: a grid launched behind this one (the decode
       // kernel) may take SMs as this kernel's CTAs leave
       if (is_k) ptx::allow_dependent_launch();
@@ -292,7 +414,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       for (int t = max(0, gt - NST); t < gt && ok; ++t) wait_or_flag(&full[t % NST], (t / NST) & 1, err, ok);
       if (is_k && un >= 1) wait_or_flag(q_full, (un - 1) & 1, err, ok);
     }
-  } else if (warp >= 9) {
+  } else if (warp == 9 || warp == 10) {
     // ---------------------------------------------------------------- MMA
     // One thread per query tile, so the two tiles' pipelines only meet at
     // the shared K/V rings: each thread walks every unit and K/V tile,
@@ -306,14 +428,18 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       const uint32_t v_addr = ptx::smem_u32(sV);
       const uint32_t col_s = C::kColS0 + t * 2 * C::BN, col_o = C::kColO0 + t * D;
       int gt = 0, un = 0, ns = 0, np = 0, nu = 0;
+      PH_DECL;
       // O_t += P_t V for the tile's next P (TMEM S buffer np & 1, bf16
       // packed, 16 keys = 8 columns per MMA step); `first` starts a unit's
       // accumulation and must wait until this tile's previous epilogue has
       // read O_t.
       auto issue_pv = [&](int vs, bool first) {
         const int l = np++, pb = l & 1;
+        PH_MARK(3);
         if (!wait_or_flag(p_full(t, pb), (l >> 1) & 1, err, ok)) return;
+        PH_MARK(4);
         if (first && nu >= 2 && !wait_or_flag(o_free(t), (nu - 2) & 1, err, ok)) return;
+        PH_MARK(5);
         ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
@@ -321,6 +447,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
           mma_bf16_ts(tmem + col_o, tmem + col_s + pb * C::BN + kk * 8, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
         }
         ptx::mma_commit(pv_done(t, pb));
+        PH_MARK(6);
       };
       for (;; ++un) {
         int u = -1;
@@ -330,6 +457,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         }
         if (u < 0 || !ok) break;
         const Unit x = load_unit(a, u, C::BN);
+        PH_MARK(0);
         const bool live = x.R > t * C::BM;
         if (!live) {
           // nothing to compute: release Q and the unit's K/V stages as they
@@ -349,6 +477,8 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
           const int ks = gt % C::KST;
           if (!wait_or_flag(&k_full[ks], (gt / C::KST) & 1, err, ok)) break;
+          PH_MARK(1);
+          PH_COUNT(7, 1);
           ptx::tc_fence_after();
           // S buffer sb holds P of this tile's tile ns - 2, which the P.V
           // issued earlier reads: the tensor core runs this thread's MMAs in
@@ -365,6 +495,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
           ptx::mma_commit(s_full(t, sb));
           ptx::mma_commit(&k_empty[ks]);
           if (i == x.n_tiles - 1) ptx::mma_commit(q_empty);
+          PH_MARK(2);
           if (i >= 1) {
             const int vs = (gt - 1) % C::VST;
             if (!wait_or_flag(&v_full[vs], ((gt - 1) / C::VST) & 1, err, ok)) break;
@@ -380,6 +511,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
           }
         }
       }
+      PH_FLUSH(true, 24 + 8 * t, 8);
     }
   } else {
     // ---------------------------------------------------- softmax / epilogue
@@ -388,6 +520,8 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t col_s = C::kColS0 + qt * 2 * C::BN, col_o = C::kColO0 + qt * D;
     int gt = 0, lt = 0, un = 0;  // global K/V tiles; tiles of this query tile; units
+    int hs = 0;                  // K/V tiles in which this warp took its exponential turn
+    PH_DECL;
     for (;; ++un) {
       int u = -1;
       if (!uq.pop(un, true, kWaitLimit, &u)) {
@@ -409,11 +543,19 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         upper = min(x.ke, p_r + 1);
       }
       const bool warp_live = qt * C::BM + (warp & 3) * 32 < x.R;
+      // this warp and its partner in the other query tile take turns when
+      // both have rows in the unit (the tile-1 warp's rows are the later ones)
+      const bool turns = C::BM + (warp & 3) * 32 < x.R;
+      uint64_t* my_turn = &turn[2 * (warp & 3) + qt];
+      uint64_t* their_turn = &turn[2 * (warp & 3) + (qt ^ 1)];
       float m_used = -INFINITY, l = 0.f;
+      PH_MARK(9);
       for (int i = 0; i < x.n_tiles && ok; ++i, ++lt, ++gt) {
         const int sb = lt & 1;
         const int k0 = x.k00 + i * C::BN;
         if (!wait_or_flag(s_full(qt, sb), (lt >> 1) & 1, err, ok)) break;
+        PH_MARK(0);
+        PH_COUNT(10, 1);
         if (warp_live) {
           ptx::tc_fence_after();
           uint32_t raw[C::BN];
@@ -422,6 +564,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
             ptx::tmem_ld32(tmem + lane_base + col_s + sb * C::BN + c * 32,
                            *reinterpret_cast<uint32_t(*)[32]>(&raw[c * 32]));
           ptx::tmem_ld_wait();
+          PH_MARK(1);
           float sv[C::BN];
           const int c_lo = lower - k0, c_hi = upper - k0;
 #pragma unroll
@@ -449,6 +592,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
             m_used = mts;
             l *= alpha;
           }
+          PH_MARK(2);
           // O may be rescaled only once the P.V of the previous tile is done
           if (i >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
             if (!wait_or_flag(pv_done(qt, (lt - 1) & 1), ((lt - 1) >> 1) & 1, err, ok)) break;
@@ -470,6 +614,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
             }
             ptx::tmem_st_wait();
           }
+          PH_MARK(3);
           // P = 2^(s*scale - m_used), packed two bf16 per 32-bit word, written
           // over the first BN/2 columns of this S buffer (lane r = row r);
           // the scale-and-shift and the running sums use the packed f32x2
@@ -479,18 +624,34 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
                           make_float2(0.f, 0.f)};
           const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
           const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(neg_m, neg_m);
+          // wait for this warp's turn: tile 0 after tile 1's previous K/V
+          // tile, tile 1 after tile 0's current one
+          PH_MARK(4);
+          if (turns && (qt == 1 || hs >= 1) &&
+              !wait_or_flag(my_turn, (qt == 1 ? hs : hs - 1) & 1, err, ok))
+            break;
+          PH_MARK(11);
           uint32_t pw[C::BN / 2];
 #pragma unroll
           for (int c = 0; c < C::BN / 2; ++c) {
             const float2 xx = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), sc2, nm2);
-            const float2 pp = make_float2(ex2(xx.x), ex2(xx.y));
+            const float2 pp = (kExp2FmaEvery > 0 && c % (kExp2FmaEvery > 0 ? kExp2FmaEvery : 1) ==
+                                                         kExp2FmaEvery - 1)
+                                  ? ex2_fma2(xx)
+                                  : make_float2(ex2(xx.x), ex2(xx.y));
             ls[c & 3] = __fadd2_rn(ls[c & 3], pp);
             __nv_bfloat162 pr = __floats2bfloat162_rn(pp.x, pp.y);
             pw[c] = *reinterpret_cast<uint32_t*>(&pr);
           }
           ptx::tmem_st32(tmem + lane_base + col_s + sb * C::BN, pw);
+          if (turns) {
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(their_turn);
+            ++hs;
+          }
           const float2 l01 = __fadd2_rn(ls[0], ls[1]), l23 = __fadd2_rn(ls[2], ls[3]);
           l += (l01.x + l01.y) + (l23.x + l23.y);
+          PH_MARK(4);
           // keys at or past the sequence end may hold anything (unwritten
           // slots, stale stage data): zero those V rows so 0 * garbage cannot
           // reach O. Both warpgroups may do it for a stage (the same zeros),
@@ -511,6 +672,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
             }
             ptx::fence_proxy_async_smem();
           }
+          PH_MARK(5);
           ptx::tmem_st_wait();
         }
         // padding warps write no P: arriving right after their s_full wait
@@ -518,6 +680,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(p_full(qt, sb));
+        PH_MARK(6);
       }
       if (!ok) break;
       // epilogue: wait for the unit's last PV, read the O row out of TMEM
@@ -525,6 +688,7 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       // O (the next unit's first P.V may start; the stores are in flight)
       const int last = lt - 1;
       if (!wait_or_flag(pv_done(qt, last & 1), (last >> 1) & 1, err, ok)) break;
+      PH_MARK(7);
       ptx::tc_fence_after();
       if (warp_live) {
         const int row = x.row0 + rr / g;
@@ -585,7 +749,9 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(o_free(qt));
+      PH_MARK(8);
     }
+    PH_FLUSH(lane == 0 && (warp & 3) == 0, 12 * qt, 12);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -593,6 +759,13 @@ __global__ void __launch_bounds__(352, 1) attn_tc_kernel(const __grid_constant__
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
+#ifdef FG_PHASE_TRACE
+  if (threadIdx.x == 0) {
+    atomicAdd(&g_phase[56], (unsigned long long)(clock64() - cta_t0));
+    atomicAdd(&g_phase[57], 1ull);
+    atomicMax(&g_phase[60], ptx::global_timer_ns());
+  }
+#endif
 }
 
 template <int D>
@@ -633,3 +806,20 @@ cudaError_t launch_attention_tc(const void* tm_q, const void* tm_kv, const Cache
 }
 
 }  // namespace fg
+
+#ifdef FG_PHASE_TRACE
+// Trace build only: copies the query-tile kernel's phase-cycle table (the
+// slot layout above g_phase) to `out` (n <= 64 entries, host memory) after
+// synchronising the device, and zeroes it when `reset` is set. 0 on success.
+extern "C" int fg_phase_trace_read(unsigned long long* out, int n, int reset) {
+  if (!out || n < 0 || n > fg::kPhaseSlots) return 1;
+  if (cudaDeviceSynchronize() != cudaSuccess) return 2;
+  if (cudaMemcpyFromSymbol(out, fg::g_phase, (size_t)n * 8) != cudaSuccess) return 2;
+  if (reset) {
+    unsigned long long init[fg::kPhaseSlots] = {};
+    init[58] = ~0ull;  // running minimum
+    if (cudaMemcpyToSymbol(fg::g_phase, init, sizeof(init)) != cudaSuccess) return 2;
+  }
+  return 0;
+}
+#endif

@@ -125,8 +125,30 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
     for (const WorkItem& w : v) P.sort_tmp[cnt[kBuckets - 1 - stages(w)]++] = w;
     v.swap(P.sort_tmp);
   };
+  // Query tiles: longest first by a coarse length (the top four bits of the
+  // 64-key stage count: units within about 6 % of each other tie), and among
+  // ties grouped by (kv head, first key, sequence). Units that read the same
+  // keys of the same kv head then run at the same time on different SMs, so
+  // their K/V tiles are fetched from DRAM about once and served from L2 to
+  // the rest; ordered by exact length alone, the concurrent units of a long
+  // prompt span every kv head and key range at once, more K/V than L2 holds.
+  auto by_length_grouped = [](std::vector<WorkItem>& v) {
+    auto coarse = [](const WorkItem& w) {
+      int n = (w.key_end - (w.key_begin - (w.key_begin & 63)) + 63) >> 6;
+      int sh = 0;
+      while ((n >> sh) >= 16) ++sh;
+      return (n >> sh) << sh;
+    };
+    std::stable_sort(v.begin(), v.end(), [&](const WorkItem& a, const WorkItem& b) {
+      const int ca = coarse(a), cb = coarse(b);
+      if (ca != cb) return ca > cb;
+      if (a.kv_head != b.kv_head) return a.kv_head < b.kv_head;
+      if (a.key_begin != b.key_begin) return a.key_begin < b.key_begin;
+      return a.seq < b.seq;
+    });
+  };
   by_length(P.decode);
-  by_length(P.tc);
+  by_length_grouped(P.tc);
   by_length(P.dtc);
   P.n_general = (int32_t)P.general.size();
   P.n_decode = (int32_t)P.decode.size();

@@ -84,7 +84,7 @@ constexpr int kConsumers = 128;
 
 // What the producer tells the consumers about a unit.
 struct UnitMeta {
-  int32_t t, h0, h1, blk, slot, pad[3];
+  int32_t t, h0, h1, blk, slot, pos, pad[2];
 };
 
 template <int D>
@@ -96,18 +96,19 @@ struct RotCfg {
   static constexpr int kMeta = kRope + HALF * 16;
   static constexpr int kStage = kMeta + (int)sizeof(UnitMeta);
   static constexpr int kBar = kStages * kStage;
-  static constexpr int kSmem = kBar + 2 * kStages * 8;
+  static constexpr int kMetaRing = kBar + 2 * kStages * 8;  // 32 UnitMeta: the producer warp's batch
+  static constexpr int kSmem = kMetaRing + 32 * (int)sizeof(UnitMeta);
 };
 
 // A unit is (token, chunk of 32 heads of the concatenated q | k | v rows).
-// Warp 4 (one lane) is the producer: for each of the CTA's units (blockIdx.x,
-// + gridDim.x, ...) it resolves the token's sequence, position and cache
-// block, writes them into the stage, and pulls the unit's rows (each of q, k
-// and v a contiguous run of whole heads) and the position's rotary row with
-// 1-D bulk copies on the stage's mbarrier. Warps 0-3 rotate from shared
-// memory and store 16-byte vectors, then free the stage. With three stages
-// the producer's dependent metadata loads and the copies stay ahead of the
-// arithmetic.
+// Warp 4 is the producer. For each batch of 32 of the CTA's units
+// (blockIdx.x, + gridDim.x, ...) its lane j resolves unit j's sequence,
+// position and cache block (a chain of dependent metadata loads; the 32
+// chains run at once) into a shared batch table; lane 0 then, stage by
+// stage, writes a unit's metadata into the stage and pulls its rows (each of
+// q, k and v a contiguous run of whole heads) and the position's rotary row
+// with 1-D bulk copies on the stage's mbarrier. Warps 0-3 rotate from shared
+// memory and store 16-byte vectors, then free the stage.
 // ROT = false: the append alone (models without rotary embedding): the head
 // list is k | v (Hq = 0) and K is copied like V.
 template <int D, bool ROT>
@@ -135,43 +136,63 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
 
   if (threadIdx.x >= kConsumers) {
     // ------------------------------------------------------------ producer
-    if (threadIdx.x != kConsumers) return;
+    const int lane = threadIdx.x - kConsumers;
+    UnitMeta* batch_meta = reinterpret_cast<UnitMeta*>(smem + C::kMetaRing);
     int it = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
-      const int st = it % kStages;
-      if (it >= kStages && !ptx::mbar_wait_bounded(&empty[st], ((it / kStages) - 1) & 1, kWaitLimit)) {
-        atomicOr(batch.err, kErrTimeout);
-        return;  // the consumers give up on the full barrier of this stage
+    bool ok = true;
+    for (int base = blockIdx.x; base < n_units && ok; base += 32 * gridDim.x) {
+      {
+        const int u = base + lane * gridDim.x;
+        UnitMeta m{};
+        m.t = -1;
+        if (u < n_units) {
+          const int t = u / chunks;
+          const int h0 = (u - t * chunks) * kChunkHeads;
+          const int s = batch.tok_seq[t];
+          const int pos = batch.ctx[s] + (t - batch.cu_q[s]);
+          const int lb = pos / cache.block_size;
+          m.t = t;
+          m.h0 = h0;
+          m.h1 = min(h0 + kChunkHeads, Hq + 2 * Hkv);
+          m.blk = batch.bt[batch.bt_off[s] + lb];
+          m.slot = pos - lb * cache.block_size;
+          m.pos = pos;
+        }
+        batch_meta[lane] = m;
       }
-      unsigned char* stage = smem + st * C::kStage;
-      const int t = u / chunks;
-      const int h0 = (u - t * chunks) * kChunkHeads;
-      const int h1 = min(h0 + kChunkHeads, Hq + 2 * Hkv);
-      const int s = batch.tok_seq[t];
-      const int pos = batch.ctx[s] + (t - batch.cu_q[s]);
-      const int lb = pos / cache.block_size;
-      UnitMeta m;
-      m.t = t;
-      m.h0 = h0;
-      m.h1 = h1;
-      m.blk = batch.bt[batch.bt_off[s] + lb];
-      m.slot = pos - lb * cache.block_size;
-      *reinterpret_cast<UnitMeta*>(stage + C::kMeta) = m;
-      const bool rot = ROT && h0 < Hq + Hkv;
-      ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((h1 - h0) * ROW + (rot ? HALF * 16 : 0)));
-      if (rot) ptx::bulk_g2s(stage + C::kRope, rope + (int64_t)pos * HALF, HALF * 16, &full[st]);
-      // [h0, h1) cut by the q, k and v ranges of the concatenated head list
-      const int qa = h0, qb = min(h1, Hq);
-      if (qa < qb)
-        ptx::bulk_g2s(stage, q + ((int64_t)t * Hq + qa) * D, (uint32_t)((qb - qa) * ROW), &full[st]);
-      const int ka = max(h0, Hq), kb = min(h1, Hq + Hkv);
-      if (ka < kb)
-        ptx::bulk_g2s(stage + (ka - h0) * ROW, k + ((int64_t)t * Hkv + (ka - Hq)) * D,
-                      (uint32_t)((kb - ka) * ROW), &full[st]);
-      const int va = max(h0, Hq + Hkv), vb = h1;
-      if (va < vb)
-        ptx::bulk_g2s(stage + (va - h0) * ROW, v + ((int64_t)t * Hkv + (va - Hq - Hkv)) * D,
-                      (uint32_t)((vb - va) * ROW), &full[st]);
+      __syncwarp();
+      if (lane == 0) {
+        for (int j = 0; j < 32; ++j, ++it) {
+          const UnitMeta m = batch_meta[j];
+          if (m.t < 0) break;
+          const int st = it % kStages;
+          if (it >= kStages && !ptx::mbar_wait_bounded(&empty[st], ((it / kStages) - 1) & 1, kWaitLimit)) {
+            atomicOr(batch.err, kErrTimeout);
+            ok = false;  // the consumers give up on the full barrier of this stage
+            break;
+          }
+          unsigned char* stage = smem + st * C::kStage;
+          *reinterpret_cast<UnitMeta*>(stage + C::kMeta) = m;
+          const int t = m.t, h0 = m.h0, h1 = m.h1, pos = m.pos;
+          const bool rot = ROT && h0 < Hq + Hkv;
+          ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((h1 - h0) * ROW + (rot ? HALF * 16 : 0)));
+          if (rot) ptx::bulk_g2s(stage + C::kRope, rope + (int64_t)pos * HALF, HALF * 16, &full[st]);
+          // [h0, h1) cut by the q, k and v ranges of the concatenated head list
+          const int qa = h0, qb = min(h1, Hq);
+          if (qa < qb)
+            ptx::bulk_g2s(stage, q + ((int64_t)t * Hq + qa) * D, (uint32_t)((qb - qa) * ROW), &full[st]);
+          const int ka = max(h0, Hq), kb = min(h1, Hq + Hkv);
+          if (ka < kb)
+            ptx::bulk_g2s(stage + (ka - h0) * ROW, k + ((int64_t)t * Hkv + (ka - Hq)) * D,
+                          (uint32_t)((kb - ka) * ROW), &full[st]);
+          const int va = max(h0, Hq + Hkv), vb = h1;
+          if (va < vb)
+            ptx::bulk_g2s(stage + (va - h0) * ROW, v + ((int64_t)t * Hkv + (va - Hq - Hkv)) * D,
+                          (uint32_t)((vb - va) * ROW), &full[st]);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();  // the batch table is rewritten only after lane 0 has read it
     }
     return;
   }

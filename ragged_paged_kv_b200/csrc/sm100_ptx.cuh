@@ -18,6 +18,13 @@ __device__ __forceinline__ int sm_id() {
   return (int)v;
 }
 
+// The global nanosecond timer (PTX %globaltimer), comparable across SMs.
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // Programmatic dependent launch: wait until the grids this one was launched
 // behind have completed and their memory is visible (a no-op for a grid
 // launched without the attribute), and let the dependent grid start once

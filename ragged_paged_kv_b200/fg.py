@@ -11,10 +11,12 @@ import re
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-# RAGGED_PAGED_KV_LIB=trace selects the instrumented build (libfg_trace.so:
-# the same kernels plus cycle accounting in the query-tile kernel)
-LIB_PATH = os.path.join(_PKG, "libfg_trace.so" if os.environ.get("RAGGED_PAGED_KV_LIB") == "trace"
-                        else "libfg.so")
+# RAGGED_PAGED_KV_LIB=<name> loads libfg_<name>.so from the package instead
+# of libfg.so: "trace" is the instrumented build (the same kernels plus cycle
+# accounting in the query-tile kernel, python -m ragged_paged_kv_b200.build
+# --trace)
+_VARIANT = os.environ.get("RAGGED_PAGED_KV_LIB", "")
+LIB_PATH = os.path.join(_PKG, f"libfg_{_VARIANT}.so" if _VARIANT else "libfg.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fg.h")
 
 STATUS = {0: "FG_OK", 1: "FG_ERR_INVALID_ARG", 2: "FG_ERR_OUT_OF_RANGE", 3: "FG_ERR_ALIAS",

@@ -7,7 +7,10 @@ whose key ranges, cut at most into pieces, exactly cover the keys that token
 may see: from max(0, p - W + 1), or 0 without a window, to its own position
 p. Each sequence must go to the kernel its shape selects. Split pieces must
 own disjoint partial rows, which their combine group lists in key order.
-Each list must be ordered longest first.
+Each list must be ordered longest first; the query-tile list by a coarse
+length (the stage count with all but its top four bits cleared) and, among
+equal coarse lengths, by (kv head, first key, sequence), so that units that
+read the same K/V run together.
 """
 import numpy as np
 import pytest
@@ -35,6 +38,12 @@ def stages(u):
     return min(4095, (int(u[KE]) - (kb - kb % 64) + 63) >> 6)
 
 
+def coarse(n):
+    """n with all but its four leading bits cleared."""
+    b = max(0, int(n).bit_length() - 4)
+    return (int(n) >> b) << b
+
+
 def check_plan(q_lens, ctx_lens, hkv, g, d, window, use_tc, slots=148):
     p = fg.describe_plan(q_lens, ctx_lens, hkv, g, d, window, use_tc, slots)
     kinds = ("general", "decode", "tc", "dtc")
@@ -46,9 +55,11 @@ def check_plan(q_lens, ctx_lens, hkv, g, d, window, use_tc, slots=148):
     for s, q in enumerate(q_lens):
         assert owner.get(s) == {expected_kernel(int(q), g, d, use_tc)}, (s, owner.get(s))
     # longest first within each persistent kernel's list
-    for kind in ("decode", "tc", "dtc"):
+    for kind in ("decode", "dtc"):
         st = [stages(u) for u in p[kind]]
         assert all(a >= b for a, b in zip(st, st[1:])), kind
+    keys = [(-coarse(stages(u)), int(u[HEAD]), int(u[KB]), int(u[SEQ])) for u in p["tc"]]
+    assert keys == sorted(keys), "tc order"
     # group the pieces by (seq, head, tile)
     tiles = {}
     for kind in kinds:
