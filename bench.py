@@ -511,36 +511,56 @@ def run_fg(args, w, rank, ws, local_rank):
     m = device_timing(fp, args.steps, args.warmup, local_rank)
     ms = m["ms"]
 
-    # end to end through the public API from pinned host buffers
-    stream, batch, cache = fp.stream, fp.batch, fp.cache
+    # end to end through the public API from pinned host buffers: each pass
+    # uploads its q, k, v and downloads its output, pipelined across passes
+    # (fg.HostPipeline: pass i + 1's upload and pass i - 1's download run
+    # while pass i computes); the window runs from the first upload to the
+    # last download, over K passes. The L2 flush still runs on the compute
+    # stream after every pass.
+    batch = fp.batch
     host_in = {n: t.cpu().pin_memory() for n, t in (("q", fp.q), ("k", fp.k), ("v", fp.v))}
     host_out = torch.empty(fp.out.shape, dtype=fp.out.dtype).pin_memory()
-    dev_bufs = {"q": fp.q, "k": fp.k, "v": fp.v, "q_rot": fp.q_rot, "out": fp.out}
+    pipe = fg.HostPipeline(fp.cache, w.n_tokens, w.n_q_heads, dev)
 
-    def e2e_step():
-        batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, stream)
-        fg.forward_host(cache, batch, host_in, dev_bufs, host_out, w.n_q_heads, w.rope_theta,
-                        w.softmax_scale, w.sliding_window, stream)
+    def e2e_submit():
+        pipe.submit(batch, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, host_in["q"], host_in["k"],
+                    host_in["v"], host_out, w.rope_theta, w.softmax_scale, w.sliding_window)
+        with torch.cuda.stream(pipe.comp):
+            fp.flush.zero_()
+            fp.flush.sum()
 
     for _ in range(max(3, args.warmup)):
-        e2e_step()
-        fp.flush_l2()
+        e2e_submit()
+    pipe.drain()
     torch.cuda.synchronize()
-    e2e_ev = [_events() for _ in range(args.steps)]
     barrier()
+    e2e_start, e2e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_start.record(pipe.up)
     for i in range(args.steps):
-        e2e_ev[i][0].record(stream)
-        e2e_step()
-        e2e_ev[i][1].record(stream)
-        fp.flush_l2()
+        e2e_submit()
+    e2e_end.record(pipe.down)
+    pipe.drain()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in e2e_ev) / args.steps, dev)
+    e2e_ms = max_over_ranks(e2e_start.elapsed_time(e2e_end) / args.steps, dev)
+    batch.device_status(pipe.comp)
+    # the link's own ceiling: the same q, k, v bytes as plain pinned
+    # host-to-device copies, back to back (no compute, no download)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(pipe.up):
+        c0.record(pipe.up)
+        for _ in range(args.steps):
+            for n in ("q", "k", "v"):
+                pipe.bufs[0][n][:w.n_tokens].copy_(host_in[n], non_blocking=True)
+        c1.record(pipe.up)
+    c1.synchronize()
+    h2d_only_ms = c0.elapsed_time(c1) / args.steps
+    qkv_bytes = sum(t.numel() * 2 for t in host_in.values())
     meta_bytes = 4 * (3 * w.n_seqs + 2 + w.n_tokens +
                       sum(w.blocks_used(s) for s in range(w.n_seqs)))
     h2d = sum(t.numel() * 2 for t in host_in.values()) + meta_bytes
     d2h = host_out.numel() * 2
-    del host_in, host_out, dev_bufs
+    del host_in, host_out, pipe
     fp.close()
 
     # the other gated configurations, measured the same way in this run
@@ -594,7 +614,11 @@ def run_fg(args, w, rank, ws, local_rank):
         "l2": "flushed between steps (256 MB write, then the same 256 MB read back; outside the events)",
         "roofline": roof,
         "e2e": {"value": tokens / (e2e_ms / 1000), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "window": "first upload to last download over K passes pipelined through fg.HostPipeline "
+                          "(upload of pass i+1 and download of pass i-1 overlap pass i), divided by K",
+                "h2d_copy_only_ms_per_step": h2d_only_ms,
+                "h2d_copy_only_GBps": qkv_bytes / (h2d_only_ms / 1000) / 1e9},
         "gpu_launches": launches,
         "plan": dict(m["info"], overlap=args.overlap),
         "clocks": m["clocks"],
@@ -604,6 +628,76 @@ def run_fg(args, w, rank, ws, local_rank):
     if ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
+    return 0
+
+
+PHASES = {
+    "softmax": ["wait_S", "load_S", "max", "rescale_O", "exp_and_store_P", "zero_V", "store_wait_and_arrive",
+                "epilogue_wait", "epilogue_store", "unit_pop", None, "turn_wait"],
+    "mma": ["unit_pop", "wait_K", "issue_S", "wait_V", "wait_P", "wait_O_free", "issue_PV"],
+    "loader": ["unit_pop", "wait_Q_free", "wait_stage_free", "issue"],
+}
+
+
+def run_phase_trace(args, w):
+    """Cycle accounting of the query-tile kernel's roles (the trace build,
+    RAGGED_PAGED_KV_LIB=trace): the same steps as the bench, then one JSON
+    line with, per role, the SM cycles spent in each phase summed over the
+    CTAs and divided by the role's 64-key tiles, the mean kernel cycles per
+    CTA, and per launch its event-timed duration beside the span from the
+    first CTA's start to the last CTA's end (%globaltimer) and the spread of
+    the CTA start times. Not a timing run: the marks themselves cost cycles,
+    and the steps run without programmatic dependent launch (per-kernel
+    events are on)."""
+    import ctypes
+    import torch
+    from ragged_paged_kv_b200 import fg
+    L = fg.lib()
+    if not hasattr(L, "fg_phase_trace_read"):
+        raise SystemExit("--phase-trace needs the trace build: python -m ragged_paged_kv_b200.build --trace "
+                         "and RAGGED_PAGED_KV_LIB=trace")
+    dev = torch.device("cuda", 0)
+    fp = FgPass(w, dev)
+    for _ in range(args.warmup):
+        fp.step(_events())
+        fp.flush_l2()
+    buf = (ctypes.c_ulonglong * 64)()
+    assert L.fg_phase_trace_read(buf, 64, 1) == 0
+    # one launch per read: the table's timer slots then describe that launch;
+    # the library's events give the same launch's duration on its stream
+    fp.batch.set_timing(True)
+    tot = [0] * 64
+    spans = {"event_ms": [], "first_to_last_end_ms": [], "cta_start_skew_ms": []}
+    for _ in range(args.steps):
+        fp.step(_events())
+        kms = fp.batch.kernel_ms()
+        assert L.fg_phase_trace_read(buf, 64, 1) == 0
+        tot = [a + b for a, b in zip(tot, list(buf))]
+        spans["event_ms"].append(kms["tc"])
+        spans["first_to_last_end_ms"].append((buf[60] - buf[58]) / 1e6)
+        spans["cta_start_skew_ms"].append((buf[59] - buf[58]) / 1e6)
+        fp.flush_l2()
+    fp.batch.set_timing(False)
+    v = tot
+    out = {"kind": "phase_trace", "workload": w.name, "steps": args.steps,
+           "ctas_per_launch": v[57] / args.steps, "cycles_per_cta": v[56] / max(1, v[57]),
+           "launch_ms": {k: sum(x) / len(x) for k, x in spans.items()}}
+    for t in range(2):
+        base = 12 * t
+        n = max(1, v[base + 10])
+        out[f"softmax_tile{t}"] = {"tiles": v[base + 10],
+                                   "cycles_per_tile": {k: v[base + i] / n for i, k in enumerate(PHASES["softmax"])
+                                                       if k}}
+        base = 24 + 8 * t
+        n = max(1, v[base + 7])
+        out[f"mma_tile{t}"] = {"tiles": v[base + 7],
+                               "cycles_per_tile": {k: v[base + i] / n for i, k in enumerate(PHASES["mma"])}}
+    for name, base in (("loader_K", 40), ("loader_V", 48)):
+        n = max(1, v[base + 4])
+        out[name] = {"tiles": v[base + 4],
+                     "cycles_per_tile": {k: v[base + i] / n for i, k in enumerate(PHASES["loader"])}}
+    print(json.dumps(out), flush=True)
+    fp.close()
     return 0
 
 
@@ -779,7 +873,8 @@ def run_serve_sim(args, policy="greedy"):
     through the API, chunk by chunk. Each iteration's device time (CUDA
     events) advances a clock; a request arrives when it becomes active, gets
     its first token at the end of the iteration that completes its prompt
-    and one more at the end of every later iteration. One JSON line (kind
+    and one more at the end of every later iteration; a device spin queued
+    ahead of each pass keeps a host pause out of its events. One JSON line (kind
     "serve_sim"): throughput, percentiles of time to first token and of the
     mean time per output token, and the requests per second that meet the
     latency targets (--sla-ttft-ms, --sla-tpot-ms). `policy` is the
@@ -804,8 +899,9 @@ def run_serve_sim(args, policy="greedy"):
     scale = 1.0 / d ** 0.5
     # start-up work a server does once, outside the loop: the rotary table
     # for the longest context (prompts stay below 8192 tokens here), and one
-    # untimed pass through the first iterations, so that module loading,
-    # launch set-up and the first growth of the plan buffers are not counted
+    # untimed pass through the whole schedule, so that module loading, launch
+    # set-up and the growth of the batch's staging and plan buffers to the
+    # largest pass (a server sizes them once) are not counted
     cache.prepare_rotary(10000.0, 8191)
 
     def one_pass(bt, alloc_):
@@ -818,6 +914,12 @@ def run_serve_sim(args, policy="greedy"):
             tab[i, :len(t)] = t
         T = int(ql.sum())
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # about 1 ms of device spin ahead of the pass, so that the device is
+        # still busy while the host validates and enqueues it: the events then
+        # time the device's work, not a pause of the host (a garbage
+        # collection, a page fault) between them
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(2_000_000)
         e0.record(stream)
         batch.put(cache, rids, ql, cl, tab, stream)
         fg.rotary_kv_append(cache, batch, q[:T], k[:T], v[:T], q_rot[:T], Hq, 10000.0, stream)
@@ -827,9 +929,13 @@ def run_serve_sim(args, policy="greedy"):
         return T, e0.elapsed_time(e1)
 
     warm_alloc = BlockAllocator(n_blocks, B, seed=1)
-    for it, bt in W.splitfuse_schedule(seed=2, budget=budget, policy=policy):
-        if it >= 64:
-            break
+    warm_events = []
+    warm_seen = 0
+    for it, bt in W.splitfuse_schedule(seed=2, budget=budget, policy=policy, events=warm_events):
+        for _, _, _, left in warm_events[warm_seen:]:
+            for r in left:
+                warm_alloc.release(r)
+        warm_seen = len(warm_events)
         one_pass(bt, warm_alloc)
     torch.cuda.synchronize()
 
@@ -905,6 +1011,8 @@ def main():
                     help="size the block pool to what the batch uses (small ncu captures)")
     ap.add_argument("--qkv-fused", action="store_true",
                     help="time the fused Q/K/V projection + rotary + append and the output projection (one GPU; JSON lines, no contract line)")
+    ap.add_argument("--phase-trace", action="store_true",
+                    help="cycle accounting of the query-tile kernel's roles (trace build; JSON line, no contract line)")
     ap.add_argument("--serve-sim", action="store_true",
                     help="timed SplitFuse loop with closed-loop synthetic clients (one GPU; JSON line)")
     ap.add_argument("--policy", choices=["greedy", "equal_split", "both"], default="both",
@@ -928,6 +1036,8 @@ def main():
     w = make_workload(args.config, args.compact_pool, world()[2], gpu=args.impl == "fg")
     if args.qkv_fused:
         return run_qkv_fused(args, w)
+    if args.phase_trace:
+        return run_phase_trace(args, w)
     if args.impl == "reference":
         rank, ws = init_dist("gloo")
         rc = run_reference(args, w, rank, ws)
