@@ -28,7 +28,10 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
   P.max_combine_rows = 0;
   const int tok_per_tile = std::max(1, kGeneralRows / g);
   const int S = (int)q_lens.size();
-  int dense_split = 0;  // pieces per long query tile, decided on first use
+  // Pieces per dense query tile (the same for all kv heads of a token tile),
+  // in emit order; decided before emitting (see below).
+  std::vector<int32_t>& dense_pieces = P.sort_tmp_pieces;
+  dense_pieces.clear();
   // Append the units of one (seq, token tile) over keys [kb, ke) for every kv
   // head to `list`, split on `split`-key boundaries of absolute position.
   // The split ranges are computed once and repeated per head.
@@ -58,6 +61,52 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
     }
     P.max_combine_rows = std::max(P.max_combine_rows, R);
   };
+  // Few long query tiles leave persistent CTAs idle at the end. The target
+  // is about 4 units per CTA slot: when the dense tiles (x kv heads) are
+  // fewer, the longest tiles of at least 2 * kTcMinSplitKeys keys are cut
+  // into pieces of at least kTcMinSplitKeys keys, merged by the combine
+  // kernel, and only as many as the target needs: P pieces per kv head are
+  // spread over the n cut-able tiles as floor(P / n) each, one more for the
+  // P % n longest (at most 8 per tile). Splitting only what the balance
+  // needs keeps the split partials, which are written in fp32 and merged
+  // again, few.
+  size_t dense_next = 0;
+  if (use_tc) {
+    const int tpt = kTcUnitRows / g;
+    std::vector<std::pair<int32_t, int32_t>> elig;  // (keys, index in emit order)
+    int32_t n_tiles = 0, n_inelig = 0;
+    for (int s = 0; s < S; ++s) {
+      const int q = q_lens[s], c = ctx_lens[s];
+      // the sequences the loop below sends to the decode kernels
+      if (q == 1 && ((head_dim == 128 && g <= kDtcMaxGroup) || g == 1)) continue;
+      for (int t0 = 0; t0 < q; t0 += tpt, ++n_tiles) {
+        const int nt = std::min(tpt, q - t0);
+        const int p0 = c + t0, p1 = c + t0 + nt - 1;
+        const int kb = window > 0 ? std::max(0, p0 - window + 1) : 0;
+        const int nk = p1 + 1 - kb;
+        if (nt * g > 16 && nk >= 2 * kTcMinSplitKeys)
+          elig.push_back({nk, n_tiles});
+        else
+          ++n_inelig;
+      }
+    }
+    const long long target = 4LL * slots;
+    if (!elig.empty() && (long long)n_tiles * n_kv_heads < target) {
+      const long long per_head = (target + n_kv_heads - 1) / n_kv_heads;  // pieces per kv head
+      const long long pe = per_head - n_inelig;                            // for the cut-able tiles
+      const long long n = (long long)elig.size();
+      const long long base = pe / n, rem = pe % n;
+      if (base >= 1) {
+        std::stable_sort(elig.begin(), elig.end(),
+                         [](const std::pair<int32_t, int32_t>& x, const std::pair<int32_t, int32_t>& y) {
+                           return x.first > y.first;
+                         });
+        dense_pieces.assign(n_tiles, 1);
+        for (long long i = 0; i < n; ++i)
+          dense_pieces[elig[i].second] = (int32_t)std::min<long long>(8, base + (i < rem ? 1 : 0));
+      }
+    }
+  }
   for (int s = 0; s < S; ++s) {
     const int q = q_lens[s], c = ctx_lens[s];
     if (use_tc && q == 1 && head_dim == 128 && g <= kDtcMaxGroup) {
@@ -72,26 +121,15 @@ void build_plan(const std::vector<int32_t>& q_lens, const std::vector<int32_t>& 
     }
     if (use_tc) {
       const int tpt = kTcUnitRows / g;
-      // Few long query tiles leave persistent CTAs idle at the end: then
-      // tiles of >= 2 * kTcMinSplitKeys keys are cut into pieces of at least
-      // kTcMinSplitKeys keys so that there are about 4 units per CTA slot.
-      if (dense_split == 0) {
-        long long n_dense = 0;
-        for (int s2 = 0; s2 < S; ++s2)
-          if (!(q_lens[s2] == 1 && head_dim == 128 && g <= kDtcMaxGroup))
-            n_dense += (q_lens[s2] + tpt - 1) / tpt;
-        n_dense *= n_kv_heads;
-        dense_split = n_dense > 0 && n_dense < 4LL * slots ? (int)((4LL * slots + n_dense - 1) / n_dense) : 1;
-        dense_split = std::min(dense_split, 8);
-      }
       for (int t0 = 0; t0 < q; t0 += tpt) {
         const int nt = std::min(tpt, q - t0);
         const int p0 = c + t0, p1 = c + t0 + nt - 1;
         const int kb = window > 0 ? std::max(0, p0 - window + 1) : 0;
         int split = nt * g <= 16 ? kTcDecodeSplitKeys : (1 << 30);
         const int nk = p1 + 1 - kb;
-        if (nt * g > 16 && dense_split > 1 && nk >= 2 * kTcMinSplitKeys)
-          split = std::max(kTcMinSplitKeys, ((nk + dense_split - 1) / dense_split + 63) & ~63);
+        const int pieces = dense_pieces.empty() ? 1 : dense_pieces[dense_next++];
+        if (nt * g > 16 && pieces > 1)
+          split = std::max(kTcMinSplitKeys, ((nk + pieces - 1) / pieces + 63) & ~63);
         emit(P.tc, s, t0, nt, kb, p1 + 1, split);
       }
       continue;

@@ -27,6 +27,7 @@ struct Plan {
   std::vector<CombineItem> combine;
   std::vector<WorkItem> sort_tmp;  // scratch of the longest-first sort
   std::vector<int32_t> sort_count;
+  std::vector<int32_t> sort_tmp_pieces;  // scratch: pieces per dense query tile
   int32_t part_rows = 0;         // partial rows the split units write
   int32_t max_combine_rows = 0;  // largest n_rows among combine items
   // packed device layout (bytes from the plan buffer's start)

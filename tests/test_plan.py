@@ -151,6 +151,26 @@ def test_one_long_prompt_is_split_for_the_persistent_grid():
         assert all(u[KE] - u[KB] >= 4096 for u in pieces[:-1])
 
 
+def test_only_the_longest_tiles_are_split_to_the_balance_target():
+    """The long-prompt batch (2048 new tokens at context 30720, 64/8 heads):
+    64 token tiles x 8 kv heads = 512 dense tiles for 148 CTA slots, whose
+    target is 4 units per slot (592). The planner cuts only the 10 longest
+    token tiles (the chunk's last, with the most keys) in two, for 592 units,
+    instead of every tile."""
+    w = W.config5()
+    p = check_plan(w.q_lens, w.ctx_lens, 8, 8, 128, 0, True)
+    tc = p["tc"]
+    assert len(tc) == 592
+    pieces = {}
+    for u in tc:
+        if int(u[SEQ]) == 0:
+            pieces.setdefault((int(u[HEAD]), int(u[TOK0])), []).append(u)
+    split = sorted({t0 for (h, t0), us in pieces.items() if len(us) > 1})
+    assert split == [2016 - 32 * i for i in range(10)][::-1]
+    assert all(len(us) == 2 for (h, t0), us in pieces.items() if t0 in split)
+    assert len(pieces) == 64 * 8
+
+
 def test_bad_arguments_are_rejected():
     with pytest.raises(fg.FgError):
         fg.describe_plan([0], [5], 1, 1, 128)
