@@ -117,7 +117,7 @@ def algorithmic_work(w):
 # since. Summaries with the commands are in profiles/.
 NCU_TRAFFIC = {
     2: {"decode": 1264564480, "tc": 52672512},
-    5: {"tc": 395085568},
+    5: {"tc": 421313280},
 }
 
 
