@@ -54,9 +54,16 @@ struct QkvArgs {
   int n_out;
 };
 
-// float64 -> bf16 with one rounding (truncate to float, force the last bit on
-// when anything was dropped: round to odd, then round to nearest even).
+// float64 -> bf16 with one rounding. Finite values: one PTX conversion
+// (cvt.rn.bf16.f64, round to nearest even). Others: truncate to float and
+// force the last bit on when anything was dropped (round to odd), then
+// round to nearest even, which also rounds once.
 __device__ __forceinline__ unsigned short f64_to_bf16(double x) {
+  if (isfinite(x)) {
+    unsigned short r;
+    asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(x));
+    return r;
+  }
   float f = __double2float_rz(x);
   if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
