@@ -332,6 +332,8 @@ class FgPass:
         self.q_rot, self.out = torch.empty_like(self.q), torch.empty_like(self.q)
         self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
         self.host_parts = {"put": 0.0, "append": 0.0, "attention": 0.0}
+        # fused: one fg_rotary_kv_attention call instead of the two calls
+        self.fused = False
         torch.cuda.synchronize()
 
     def step(self, ev):
@@ -342,6 +344,16 @@ class FgPass:
         self.batch.put(self.cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables, st)
         t1 = time.perf_counter()
         ev[3].record(st)
+        if self.fused:
+            t2 = time.perf_counter()
+            ev[1].record(st)
+            fg.rotary_kv_attention(self.cache, self.batch, self.q, self.k, self.v, self.q_rot, self.out,
+                                   w.n_q_heads, w.rope_theta, w.softmax_scale, w.sliding_window, st)
+            t3 = time.perf_counter()
+            ev[2].record(st)
+            self.host_parts["put"] += t1 - t0
+            self.host_parts["attention"] += t3 - t2
+            return
         fg.rotary_kv_append(self.cache, self.batch, self.q, self.k, self.v, self.q_rot, w.n_q_heads,
                             w.rope_theta, st)
         t2 = time.perf_counter()
@@ -447,6 +459,32 @@ def device_timing(fp, steps, warmup, local_rank):
             "info": info, "clocks": clocks.summary()}
 
 
+def fused_timing(fp, steps, warmup, local_rank):
+    """The same step through fg_rotary_kv_attention (one call: rotary +
+    append + attention, the query tiles' Q rotated in the query-tile
+    kernel's load): W untimed steps, then K timed steps, CUDA events on the
+    launching stream around each step, L2 flushed before each step outside
+    the events; the max over ranks of each rank's mean (ms)."""
+    import torch
+    fp.fused = True
+    for _ in range(warmup):
+        fp.step(_events())
+        fp.flush_l2()
+    torch.cuda.synchronize()
+    evs = [_events() for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        for _ in range(16 if i == 0 else 1):
+            fp.flush_l2()
+        fp.step(evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    fp.fused = False
+    fp.batch.device_status(fp.stream)
+    return max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in evs) / steps, fp.dev)
+
+
 def roofline_of(w, config, m):
     """The `roofline` object for the dominant kernel of workload w (the one
     with the longest average launch), from the measurements `m`."""
@@ -510,6 +548,7 @@ def run_fg(args, w, rank, ws, local_rank):
     fp = FgPass(w, dev, args.overlap)
     m = device_timing(fp, args.steps, args.warmup, local_rank)
     ms = m["ms"]
+    fused_ms = fused_timing(fp, args.steps, args.warmup, local_rank)
 
     # end to end through the public API from pinned host buffers: each pass
     # uploads its q, k, v and downloads its output, pipelined across passes
@@ -588,7 +627,7 @@ def run_fg(args, w, rank, ws, local_rank):
     # the other gated configurations, measured the same way in this run
     # (fewer steps), one object each under "per_config"
     per_config = {}
-    launches = args.steps * (1 + m["info"]["launches"])
+    launches = 2 * args.steps * (1 + m["info"]["launches"])
     if not args.no_per_config:
         for c in sorted(GATES):
             if c == args.config:
@@ -596,6 +635,7 @@ def run_fg(args, w, rank, ws, local_rank):
             wc = make_workload(c, args.compact_pool, local_rank)
             fpc = FgPass(wc, dev, args.overlap)
             mc = device_timing(fpc, args.per_config_steps, 3, local_rank)
+            mc_fused = fused_timing(fpc, args.per_config_steps, 3, local_rank)
             fpc.close()
             rc = roofline_of(wc, c, mc)
             bound, gate = GATES[c]
@@ -610,8 +650,8 @@ def run_fg(args, w, rank, ws, local_rank):
                 "kernel_ms": rc["kernel_ms"], "tc_TFLOPs": rc["tc_TFLOPs"],
                 "step_roofline_ms": rc["step_roofline_ms"], "step_frac": rc["step_frac"],
                 "gate": {"bound": bound, "min_frac": gate, "met": rc["bound"] == bound and rc["frac"] >= gate},
-                "clocks": mc["clocks"]}
-            launches += args.per_config_steps * (1 + mc["info"]["launches"])
+                "clocks": mc["clocks"], "fused_q_rope_ms_per_step": mc_fused}
+            launches += 2 * args.per_config_steps * (1 + mc["info"]["launches"])
 
     if rank != 0:
         return 0
@@ -643,6 +683,11 @@ def run_fg(args, w, rank, ws, local_rank):
                 "h2d_copy_only_ms_per_step": h2d_only_ms,
                 "h2d_copy_only_GBps": qkv_bytes / (h2d_only_ms / 1000) / 1e9,
                 "copies_both_directions_ms_per_step": both_ms},
+        "fused_q_rope": {"ms_per_step": fused_ms, "value": tokens / (fused_ms / 1000), "unit": "tokens/s",
+                         "entry": "fg_rotary_kv_attention",
+                         "what": "the same pass in one call: the query-tile kernel reads its Q rows unrotated and "
+                                 "rotates them in shared memory, the rotary kernel skips them; outputs and cache "
+                                 "bit-identical to the two calls timed in value"},
         "gpu_launches": launches,
         "plan": dict(m["info"], overlap=args.overlap),
         "clocks": m["clocks"],

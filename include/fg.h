@@ -217,6 +217,27 @@ fg_status fg_ragged_attention(const fg_kv_cache* cache, fg_ragged_batch* batch, 
                               void* out, int32_t n_q_heads, float softmax_scale,
                               int32_t sliding_window, void* stream);
 
+/* Steps 1 to 3 in one call: fg_rotary_kv_append followed by
+ * fg_ragged_attention, with the rotation of the queries that the query-tile
+ * (prefill) kernel serves moved into that kernel's load of Q. Those Q rows
+ * are read unrotated from q and rotated in shared memory with the same exact
+ * arithmetic and table, so the rotated Q never makes a round trip through
+ * HBM (the rotation of "DeepSpeed-FastGen — paper by Holmes et al. (2024)",
+ * Key points, as in fg_rotary_kv_append; the attention as in
+ * fg_ragged_attention). q: device [T][n_q_heads][d], not modified; k, v:
+ * device [T][Hkv][d]; q_rot: device [T][n_q_heads][d], receives the rotated
+ * rows of the tokens served by the decode kernels only (the other rows are
+ * left as they were); out: device [T][n_q_heads][d]. Every word of out and
+ * of the cache equals that of the two calls in sequence. All pointers
+ * 16-byte aligned, q_rot distinct from q. Where the query-tile kernel does
+ * not serve the batch (a group size it does not take), the call runs the
+ * two steps unchanged. Errors, allocation and ordering as the two calls;
+ * asynchronous on `stream`. */
+fg_status fg_rotary_kv_attention(fg_kv_cache* cache, fg_ragged_batch* batch, const void* q, const void* k,
+                                 const void* v, void* q_rot, void* out, int32_t n_q_heads,
+                                 double rope_theta, float softmax_scale, int32_t sliding_window,
+                                 void* stream);
+
 /* The same pass as fg_ragged_attention, for callers that must not allocate.
  * The pages have no counterpart: this is a library convenience. Some callers
  * cannot call cudaMalloc (or cudaMallocAsync / cudaFree, or a framework

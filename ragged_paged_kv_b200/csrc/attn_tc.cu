@@ -45,6 +45,7 @@
 #include <cfloat>
 
 #include "fg_internal.h"
+#include "rope_exact.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fg {
@@ -111,8 +112,9 @@ struct TcCfg {
   static constexpr int kOffBar = kOffV + VST * kKVBytes;
   // q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST],
   // then per query tile: s_full[2], p_full[2], pv_done[2], o_free; the
-  // exponential turns of the 4 softmax warp pairs (turn[2 r + t]); unit queue
-  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + NQ * 7 + 8 + 2 * UnitQueue::kDepth;
+  // exponential turns of the 4 softmax warp pairs (turn[2 r + t]); unit
+  // queue; q_ready (Q rotated in place, the rotary-at-load form)
+  static constexpr int kNumBars = 2 + 2 * KST + 2 * VST + NQ * 7 + 8 + 2 * UnitQueue::kDepth + 1;
   static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + UnitQueue::kDepth * 4;
   static constexpr int kThreads = 384;  // 8 softmax warps, the K loader, two MMA warps, the V loader
   static constexpr uint32_t kTmemCols = 512;
@@ -137,6 +139,10 @@ struct TcArgs {
   int n_items;
   int* counter;  // next-unit counter, zero at launch
   int sm_end;    // only CTAs on SMs with id < sm_end take units (the others leave at once)
+  // the rotary-at-load form (ROPE = true): Q is read unrotated and rotated
+  // in shared memory with this table ([position][d/2] (cos, sin) times
+  // 2^896, pair 8 j + e at entry e * d/16 + j)
+  const double2* rope;
 };
 
 // What every role needs to know about one unit.
@@ -233,7 +239,7 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int
   return ok;
 }
 
-template <int D>
+template <int D, bool ROPE>
 __global__ void __launch_bounds__(384, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                         const __grid_constant__ CUtensorMap tm_kv,
                                                         TcArgs a) {
@@ -277,6 +283,7 @@ __global__ void __launch_bounds__(384, 1) attn_tc_kernel(const __grid_constant__
   uint64_t* turn = tb + 7 * C::NQ;
   uint64_t* uq_full = turn + 8;
   uint64_t* uq_empty = uq_full + UnitQueue::kDepth;
+  uint64_t* q_ready = uq_empty + UnitQueue::kDepth;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   // units come from a global counter through this queue (the V loader, the
   // two MMA threads and the eight softmax warps consume)
@@ -307,6 +314,7 @@ __global__ void __launch_bounds__(384, 1) attn_tc_kernel(const __grid_constant__
       ptx::mbar_init(o_free(t), 4);
     }
     for (int i = 0; i < 8; ++i) ptx::mbar_init(&turn[i], 1);
+    ptx::mbar_init(q_ready, 8);
     uq.init();
     ptx::fence_mbar_init();
   }
@@ -473,7 +481,7 @@ __global__ void __launch_bounds__(384, 1) attn_tc_kernel(const __grid_constant__
           continue;
         }
         ++nu;
-        if (!wait_or_flag(q_full, un & 1, err, ok)) break;
+        if (!wait_or_flag(ROPE ? q_ready : q_full, un & 1, err, ok)) break;
         for (int i = 0; i < x.n_tiles && ok; ++i, ++gt) {
           const int ks = gt % C::KST;
           if (!wait_or_flag(&k_full[ks], (gt / C::KST) & 1, err, ok)) break;
@@ -530,6 +538,37 @@ __global__ void __launch_bounds__(384, 1) attn_tc_kernel(const __grid_constant__
       }
       if (u < 0 || !ok) break;
       const Unit x = load_unit(a, u, C::BN);
+      if (ROPE) {
+        // the rotary-at-load form: each thread rotates its own row of the
+        // unit's Q tile in shared memory (pairs (i, i + d/2) share a row and
+        // a swizzled 16-byte position: the two 64-dim halves at d = 128,
+        // 16-byte chunks j and j + 4 at d = 64), with the same exact
+        // arithmetic as the rotary kernel; every softmax warp arrives on
+        // q_ready once it is done (rows past the unit are left alone)
+        if (!wait_or_flag(q_full, un & 1, err, ok)) break;
+        const int rq = qt * C::BM + r;
+        if (rq < x.R) {
+          constexpr int HALF = D / 2, GROUPS = HALF / 8, NCH = HALF / 8;
+          const double2* rrow = a.rope + (int64_t)(x.ctx + x.tok_begin + rq / g) * HALF;
+          unsigned char* qrow = sQ + qt * C::kQBytes + r * 128;
+          const int sw = r & 7;
+          // one 16-byte chunk pair at a time (a table prefetch one chunk
+          // ahead measured slower: its registers push the kernel into spills)
+#pragma unroll 1
+          for (int j = 0; j < NCH; ++j) {
+            uint4* pa = reinterpret_cast<uint4*>(qrow + ((j ^ sw) << 4));
+            uint4* pb = D == 128 ? reinterpret_cast<uint4*>(qrow + C::BM * 128 + ((j ^ sw) << 4))
+                                 : reinterpret_cast<uint4*>(qrow + (((j + 4) ^ sw) << 4));
+            uint4 y1, y2;
+            rope::rotate8(*pa, *pb, [&](int e) { return __ldg(rrow + e * GROUPS + j); }, y1, y2);
+            *pa = y1;
+            *pb = y2;
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(q_ready);
+      }
       if (x.R <= qt * C::BM) {  // this query tile has no rows in the unit
         gt += x.n_tiles;
         continue;
@@ -768,23 +807,23 @@ __global__ void __launch_bounds__(384, 1) attn_tc_kernel(const __grid_constant__
 #endif
 }
 
-template <int D>
+template <int D, bool ROPE>
 cudaError_t launch_tc_d(const CUtensorMap& tm_q, const CUtensorMap& tm_kv, const TcArgs& args, int grid,
                         cudaStream_t stream) {
   using C = TcCfg<D>;
   // per device: the attributes apply to the current device only
   static PerDeviceOnce configured;
   cudaError_t e0 = configured.run([] {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     // the largest shared-memory carveout, so CTAs of different kernels can
     // share an SM
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+      e = cudaFuncSetAttribute(attn_tc_kernel<D, ROPE>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                cudaSharedmemCarveoutMaxShared);
     return e;
   });
   if (e0 != cudaSuccess) return e0;
-  attn_tc_kernel<D><<<grid, C::kThreads, C::kSmem, stream>>>(tm_q, tm_kv, args);
+  attn_tc_kernel<D, ROPE><<<grid, C::kThreads, C::kSmem, stream>>>(tm_q, tm_kv, args);
   return cudaGetLastError();
 }
 
@@ -794,15 +833,19 @@ cudaError_t launch_attention_tc(const void* tm_q, const void* tm_kv, const Cache
                                 const BatchView& batch, const WorkItem* items, int n_items,
                                 __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
                                 int g, float scale_log2, int window, int grid, int sm_end,
-                                int* counter, cudaStream_t stream) {
+                                int* counter, cudaStream_t stream, const double2* rope) {
   if (n_items == 0) return cudaSuccess;
   TcArgs args{cache, batch, items, out, part_o, part_ml, n_q_heads, g, scale_log2, window, n_items,
-              counter, sm_end};
+              counter, sm_end, rope};
   grid = grid < 1 ? 1 : (grid > n_items ? n_items : grid);
   const CUtensorMap& q = *static_cast<const CUtensorMap*>(tm_q);
   const CUtensorMap& kv = *static_cast<const CUtensorMap*>(tm_kv);
-  if (cache.head_dim == 128) return launch_tc_d<128>(q, kv, args, grid, stream);
-  return launch_tc_d<64>(q, kv, args, grid, stream);
+  if (rope) {
+    if (cache.head_dim == 128) return launch_tc_d<128, true>(q, kv, args, grid, stream);
+    return launch_tc_d<64, true>(q, kv, args, grid, stream);
+  }
+  if (cache.head_dim == 128) return launch_tc_d<128, false>(q, kv, args, grid, stream);
+  return launch_tc_d<64, false>(q, kv, args, grid, stream);
 }
 
 }  // namespace fg

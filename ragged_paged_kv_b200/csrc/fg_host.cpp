@@ -844,7 +844,7 @@ struct FixedPassStorage {
 
 fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot, void* out,
                               int32_t n_q_heads, float softmax_scale, int32_t window, cudaStream_t strm,
-                              const FixedPassStorage* fixed);
+                              const FixedPassStorage* fixed, const void* q_tc = nullptr);
 
 extern "C" fg_status fg_ragged_attention(const fg_kv_cache* c, fg_ragged_batch* b,
                                          const void* q_rot, void* out, int32_t n_q_heads,
@@ -852,6 +852,41 @@ extern "C" fg_status fg_ragged_attention(const fg_kv_cache* c, fg_ragged_batch* 
                                          void* stream) {
   return fg_attention_launch(c, b, q_rot, out, n_q_heads, softmax_scale, sliding_window,
                              static_cast<cudaStream_t>(stream), nullptr);
+}
+
+// Rotary + append + attention in one call, with the rotation of the Q rows
+// the query-tile kernel serves moved into that kernel's Q load: the rotary
+// kernel leaves those rows of q_rot unwritten (and does not read them from
+// q), and the query-tile kernel reads them unrotated from q and rotates them
+// in shared memory with the same exact arithmetic. Every output and cache
+// word equals that of fg_rotary_kv_append followed by fg_ragged_attention.
+extern "C" fg_status fg_rotary_kv_attention(fg_kv_cache* c, fg_ragged_batch* b, const void* q,
+                                            const void* k, const void* v, void* q_rot, void* out,
+                                            int32_t n_q_heads, double rope_theta, float softmax_scale,
+                                            int32_t sliding_window, void* stream) {
+  fg_status st = check_pass(c, b, n_q_heads);
+  if (st) return st;
+  if (!(rope_theta > 0.0)) return fail(FG_ERR_INVALID_ARG, "rope_theta must be > 0");
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(FG_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (sliding_window < 0) return fail(FG_ERR_INVALID_ARG, "sliding_window %d < 0", sliding_window);
+  if (b->n_tokens == 0) return FG_OK;
+  if (!q || !k || !v || !q_rot || !out) return fail(FG_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_rot) || !aligned16(out))
+    return fail(FG_ERR_INVALID_ARG, "q, k, v, q_rot and out must be 16-byte aligned");
+  if (q == q_rot) return fail(FG_ERR_INVALID_ARG, "q_rot must be distinct from q");
+  const int32_t g = n_q_heads / c->n_kv_heads;
+  const bool fuse = tc_eligible(c, g);
+  st = ensure_rope(c, rope_theta, b->max_pos);
+  if (st) return st;
+  const cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t e = fg::launch_rotary_append(
+      cache_view(c), b->view, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(q_rot), c->rope, n_q_heads, true, strm,
+      fuse ? fg::kDtcMaxGroup : 0);
+  if (e != cudaSuccess) return cuda_fail(e, "rotary_append launch");
+  return fg_attention_launch(c, b, q_rot, out, n_q_heads, softmax_scale, sliding_window, strm, nullptr,
+                             fuse ? q : nullptr);
 }
 
 // The one launch sequence of both attention entry points. With fixed ==
@@ -864,7 +899,7 @@ extern "C" fg_status fg_ragged_attention(const fg_kv_cache* c, fg_ragged_batch* 
 // storage differs; the kernels, their order and their arguments are the same.
 fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const void* q_rot, void* out,
                               int32_t n_q_heads, float softmax_scale, int32_t window, cudaStream_t strm,
-                              const FixedPassStorage* fixed) {
+                              const FixedPassStorage* fixed, const void* q_tc) {
   fg_status st = check_pass(c, b, n_q_heads);
   if (st) return st;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
@@ -879,8 +914,11 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
   if (!use_tc && g > fg::kMaxGroup)
     return fail(FG_ERR_UNSUPPORTED, "n_q_heads / n_kv_heads = %d > %d", g, fg::kMaxGroup);
   const double t_a = now_us();
+  // q_tc: the query-tile kernel reads Q unrotated from there and rotates it
+  // as it loads it (its rows of q_rot are then not needed)
+  if (q_tc && !use_tc) return fail(FG_ERR_INVALID_ARG, "rotary-at-load needs the query-tile kernel");
   CUtensorMap tm_q, tm_q1;
-  if (use_tc && (!make_q_map(&tm_q, q_rot, b->n_tokens, n_q_heads, c->head_dim, g) ||
+  if (use_tc && (!make_q_map(&tm_q, q_tc ? q_tc : q_rot, b->n_tokens, n_q_heads, c->head_dim, g) ||
                  !make_q_map(&tm_q1, q_rot, b->n_tokens, n_q_heads, c->head_dim, g, 1)))
     return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for q_rot");
   b->hprof[6] += now_us() - t_a;
@@ -970,7 +1008,7 @@ fg_status fg_attention_launch(const fg_kv_cache* c, fg_ragged_batch* b, const vo
     e = fg::launch_attention_tc(&tm_q, &c->tm_kv, cv, b->view,
                                 reinterpret_cast<const WorkItem*>(base + P.off_tc), P.n_tc, o, part_o,
                                 part_ml, n_q_heads, g, scale_log2, window, sm_count(),
-                                both ? tc_sms : INT32_MAX, ctr, tc_stream);
+                                both ? tc_sms : INT32_MAX, ctr, tc_stream, q_tc ? c->rope : nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
     if ((st = mark(1, 1, tc_stream))) return st;
   }

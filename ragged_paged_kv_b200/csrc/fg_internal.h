@@ -90,7 +90,7 @@ __host__ __device__ inline int64_t cache_offset(const CacheView& c, int64_t blk,
 cudaError_t launch_rotary_append(const CacheView& cache, const BatchView& batch,
                                  const __nv_bfloat16* q, const __nv_bfloat16* k,
                                  const __nv_bfloat16* v, __nv_bfloat16* q_rot, const double2* rope,
-                                 int n_q_heads, bool rotate, cudaStream_t stream);
+                                 int n_q_heads, bool rotate, cudaStream_t stream, int skip_tc_q = 0);
 
 cudaError_t launch_attention_general(const CacheView& cache, const BatchView& batch,
                                      const WorkItem* items, int n_items,
@@ -106,12 +106,14 @@ cudaError_t launch_attention_decode(const CacheView& cache, const BatchView& bat
 
 // tm_q / tm_kv point to CUtensorMap objects (host memory, passed by value).
 // The persistent tensor-core kernels take their units from *counter, which
-// must be zero when the kernel starts.
+// must be zero when the kernel starts. With rope != nullptr the query-tile
+// kernel reads Q unrotated (tm_q over q) and rotates it in shared memory
+// with that table (the rotary kernel's table, times 2^896).
 cudaError_t launch_attention_tc(const void* tm_q, const void* tm_kv, const CacheView& cache,
                                 const BatchView& batch, const WorkItem* items, int n_items,
                                 __nv_bfloat16* out, float* part_o, float* part_ml, int n_q_heads,
                                 int g, float scale_log2, int window, int grid, int sm_end,
-                                int* counter, cudaStream_t stream);
+                                int* counter, cudaStream_t stream, const double2* rope = nullptr);
 
 // Grouped (or MHA) one-token decode on tensor cores, keys as MMA rows;
 // tm_q1 views q_rot with boxes of 64 dims x g heads x 1 token. d = 128.

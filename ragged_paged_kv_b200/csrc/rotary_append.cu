@@ -13,65 +13,11 @@
 #include <cfloat>
 
 #include "fg_internal.h"
+#include "rope_exact.cuh"
 #include "sm100_ptx.cuh"
 
 namespace fg {
 namespace {
-
-// float64 -> bf16, round to nearest even, one rounding. Truncate to float and
-// force the last float bit on when the truncation dropped anything ("round
-// to odd", Boldo & Melquiond 2008): with 16 spare bits between float and bf16
-// the following float -> bf16 round-to-nearest-even then equals the direct
-// rounding of the double, subnormals included. Exact for every double; the
-// kernel uses it only for vectors the fast path below does not cover.
-__device__ __noinline__ unsigned short f64_to_bf16_rne_slow(double x) {
-  float f = __double2float_rz(x);
-  if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);
-  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
-}
-
-// float64 -> bf16, round to nearest even, one rounding, as one PTX
-// conversion (cvt.rn.bf16.f64). On B200 it gives the same bits as the
-// round-to-odd path above for every finite double tried (2^32 of them:
-// random bit patterns, neighbours of bf16 midpoints, the subnormal range,
-// overflow), subnormal results included.
-__device__ __forceinline__ uint32_t f64_to_bf16_cvt(double y) {
-  unsigned short r;
-  asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(y));
-  return r;
-}
-
-// A bf16 pattern widened to a double whose value is 2^-896 times the bf16's
-// value, by moving its 8 exponent bits to the low end of the double's 11-bit
-// exponent field (an arithmetic shift keeps the sign on top, the mask clears
-// the three bits in between). Exact for zero, subnormal and normal patterns;
-// infinities and NaNs are screened out per vector first. The rotary table is
-// stored times 2^896, so each product x * cos is exact and unscaled.
-__device__ __forceinline__ double bf16_lo_scaled(uint32_t w) {
-  return __hiloint2double((int)(((uint32_t)((int32_t)(w << 16) >> 3)) & 0x8FFFFFFFu), 0);
-}
-__device__ __forceinline__ double bf16_hi_scaled(uint32_t w) {
-  return __hiloint2double((int)(((uint32_t)((int32_t)w >> 3)) & 0x8FFFE000u), 0);
-}
-// Bit 15 or 31 is set iff the low or high bf16 of w has an all-ones exponent.
-__device__ __forceinline__ uint32_t special_bits(uint32_t w) {
-  return ((w & 0x7F807F80u) + 0x00800080u) & 0x80008000u;
-}
-__device__ __forceinline__ double bf16_lo(uint32_t w) { return (double)__uint_as_float(w << 16); }
-__device__ __forceinline__ double bf16_hi(uint32_t w) { return (double)__uint_as_float(w & 0xFFFF0000u); }
-
-// Rotation of one word pair (two pairs (x1, x2)) the plain way, for the
-// vectors the fast path does not cover; the table entries are times 2^896.
-__device__ __noinline__ uint2 rotate_pair_slow(uint32_t a, uint32_t b, double2 r_lo, double2 r_hi) {
-  const double x1l = bf16_lo(a), x1h = bf16_hi(a), x2l = bf16_lo(b), x2h = bf16_hi(b);
-  const double cl = r_lo.x * 0x1p-896, sl = r_lo.y * 0x1p-896;
-  const double ch = r_hi.x * 0x1p-896, sh = r_hi.y * 0x1p-896;
-  const unsigned short r1l = f64_to_bf16_rne_slow(__dsub_rn(__dmul_rn(x1l, cl), __dmul_rn(x2l, sl)));
-  const unsigned short r1h = f64_to_bf16_rne_slow(__dsub_rn(__dmul_rn(x1h, ch), __dmul_rn(x2h, sh)));
-  const unsigned short r2l = f64_to_bf16_rne_slow(__dadd_rn(__dmul_rn(x2l, cl), __dmul_rn(x1l, sl)));
-  const unsigned short r2h = f64_to_bf16_rne_slow(__dadd_rn(__dmul_rn(x2h, ch), __dmul_rn(x1h, sh)));
-  return make_uint2((uint32_t)r1l | ((uint32_t)r1h << 16), (uint32_t)r2l | ((uint32_t)r2h << 16));
-}
 
 constexpr long long kWaitLimit = 1LL << 31;
 constexpr int kChunkHeads = 32;  // heads (of q | k | v, concatenated) per unit
@@ -111,7 +57,8 @@ struct RotCfg {
 template <int D, bool ROT>
 __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_kernel(
     CacheView cache, BatchView batch, const __nv_bfloat16* q, const __nv_bfloat16* k,
-    const __nv_bfloat16* v, __nv_bfloat16* q_rot, const double2* __restrict__ rope, int Hq, int chunks) {
+    const __nv_bfloat16* v, __nv_bfloat16* q_rot, const double2* __restrict__ rope, int Hq, int chunks,
+    int skip_tc_q) {
   using C = RotCfg<D>;
   constexpr int HALF = C::HALF;
   constexpr int GROUPS = HALF / 8;  // 8-pair groups per head
@@ -151,6 +98,15 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
           m.t = t;
           m.h0 = h0;
           m.h1 = min(h0 + kChunkHeads, Hq + 2 * Hkv);
+          // Q rows the query-tile kernel rotates itself (skip_tc_q > 0: the
+          // attention call that follows reads unrotated Q for the sequences
+          // it serves, the plan's rule with skip_tc_q = the largest group the
+          // tensor-core decode kernel takes): the unit keeps its K and V
+          if (skip_tc_q > 0 && h0 < Hq) {
+            const int qn = batch.cu_q[s + 1] - batch.cu_q[s];
+            const int grp = Hq / Hkv;
+            if (!(qn == 1 && ((D == 128 && grp <= skip_tc_q) || grp == 1))) m.h0 = min(Hq, m.h1);
+          }
           m.blk = batch.bt[batch.bt_off[s] + lb];
           m.slot = pos - lb * cache.block_size;
           m.pos = pos;
@@ -171,7 +127,7 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
           unsigned char* stage = smem + st * C::kStage;
           *reinterpret_cast<UnitMeta*>(stage + C::kMeta) = m;
           const int t = m.t, h0 = m.h0, h1 = m.h1, pos = m.pos;
-          const bool rot = ROT && h0 < Hq + Hkv;
+          const bool rot = ROT && h0 < h1 && h0 < Hq + Hkv;
           ptx::mbar_arrive_expect_tx(&full[st], (uint32_t)((h1 - h0) * ROW + (rot ? HALF * 16 : 0)));
           if (rot) ptx::bulk_g2s(stage + C::kRope, rope + (int64_t)pos * HALF, HALF * 16, &full[st]);
           // [h0, h1) cut by the q, k and v ranges of the concatenated head list
@@ -226,35 +182,8 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
         const int h = m.h0 + hl;
         const uint4 a = *reinterpret_cast<const uint4*>(stage + hl * ROW + i0 * 2);
         const uint4 b = *reinterpret_cast<const uint4*>(stage + hl * ROW + (HALF + i0) * 2);
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-        uint32_t y1[4], y2[4];
-        uint32_t special = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          special |= special_bits(aw[e]) | special_bits(bw[e]);
-          const double x1l = bf16_lo_scaled(aw[e]), x1h = bf16_hi_scaled(aw[e]);
-          const double x2l = bf16_lo_scaled(bw[e]), x2h = bf16_hi_scaled(bw[e]);
-          const double cl = cs[2 * e], sl = sn[2 * e], ch = cs[2 * e + 1], sh = sn[2 * e + 1];
-          // both products are exact, so one fused multiply-add rounds the
-          // difference exactly once
-          const double r1l = __fma_rn(x1l, cl, -__dmul_rn(x2l, sl));
-          const double r1h = __fma_rn(x1h, ch, -__dmul_rn(x2h, sh));
-          const double r2l = __fma_rn(x2l, cl, __dmul_rn(x1l, sl));
-          const double r2h = __fma_rn(x2h, ch, __dmul_rn(x1h, sh));
-          y1[e] = f64_to_bf16_cvt(r1l) | (f64_to_bf16_cvt(r1h) << 16);
-          y2[e] = f64_to_bf16_cvt(r2l) | (f64_to_bf16_cvt(r2h) << 16);
-        }
-        if (special != 0u) {
-          // an infinite or NaN input: redo the vector with plain widening and
-          // the exact narrowing
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint2 r = rotate_pair_slow(aw[e], bw[e], rs[(2 * e) * GROUPS + g], rs[(2 * e + 1) * GROUPS + g]);
-            y1[e] = r.x;
-            y2[e] = r.y;
-          }
-        }
+        uint4 y1, y2;
+        rope::rotate8(a, b, [&](int e) { return make_double2(cs[e], sn[e]); }, y1, y2);
         __nv_bfloat16* dst;
         if (h < Hq) {
           dst = q_rot + ((int64_t)m.t * Hq + h) * D;
@@ -262,8 +191,8 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
           if (!blk_ok) continue;
           dst = cache.base + cache_offset(cache, m.blk, 0, h - Hq, m.slot);
         }
-        *reinterpret_cast<uint4*>(dst + i0) = make_uint4(y1[0], y1[1], y1[2], y1[3]);
-        *reinterpret_cast<uint4*>(dst + HALF + i0) = make_uint4(y2[0], y2[1], y2[2], y2[3]);
+        *reinterpret_cast<uint4*>(dst + i0) = y1;
+        *reinterpret_cast<uint4*>(dst + HALF + i0) = y2;
       }
     }
     if (blk_ok) {
@@ -291,7 +220,7 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
 cudaError_t launch_rotary_append(const CacheView& cache, const BatchView& batch,
                                  const __nv_bfloat16* q, const __nv_bfloat16* k,
                                  const __nv_bfloat16* v, __nv_bfloat16* q_rot, const double2* rope,
-                                 int n_q_heads, bool rotate, cudaStream_t stream) {
+                                 int n_q_heads, bool rotate, cudaStream_t stream, int skip_tc_q) {
   if (batch.n_tokens == 0) return cudaSuccess;
   if (!rotate) n_q_heads = 0;
   const int chunks = (n_q_heads + 2 * cache.n_kv_heads + kChunkHeads - 1) / kChunkHeads;
@@ -304,17 +233,17 @@ cudaError_t launch_rotary_append(const CacheView& cache, const BatchView& batch,
   if (cache.head_dim == 128) {
     if (rotate)
       rotary_append_kernel<128, true><<<grid, kConsumers + 32, RotCfg<128>::kSmem, stream>>>(
-          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
+          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks, skip_tc_q);
     else
       rotary_append_kernel<128, false><<<grid, kConsumers + 32, RotCfg<128>::kSmem, stream>>>(
-          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
+          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks, skip_tc_q);
   } else {
     if (rotate)
       rotary_append_kernel<64, true><<<grid, kConsumers + 32, RotCfg<64>::kSmem, stream>>>(
-          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
+          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks, skip_tc_q);
     else
       rotary_append_kernel<64, false><<<grid, kConsumers + 32, RotCfg<64>::kSmem, stream>>>(
-          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks);
+          cache, batch, q, k, v, q_rot, rope, n_q_heads, chunks, skip_tc_q);
   }
   return cudaGetLastError();
 }

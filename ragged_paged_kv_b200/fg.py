@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
         "fg_output_projection": [V, V, V, I32, I32, V, V],
         "fg_kv_cache_prepare_rotary": [V, D, I32],
         "fg_ragged_attention": [V, V, V, V, I32, F, I32, V],
+        "fg_rotary_kv_attention": [V, V, V, V, V, V, V, I32, D, F, I32, V],
         "fg_ragged_attention_noalloc": [V, V, V, V, I32, F, I32, V],
         "fg_device_status": [V, V],
         "fg_attention_plan_info": [V, _c_int32_p],
@@ -305,6 +306,18 @@ def ragged_attention(cache: KVCache, batch: RaggedBatch, q_rot, out, n_q_heads: 
                                      _dev_ptr(out, "out"), int(n_q_heads), float(softmax_scale),
                                      int(sliding_window), _stream_ptr(stream)),
            "fg_ragged_attention")
+
+
+def rotary_kv_attention(cache: KVCache, batch: RaggedBatch, q, k, v, q_rot, out, n_q_heads: int,
+                        rope_theta: float, softmax_scale: float, sliding_window: int = 0, stream=None):
+    """fg_rotary_kv_attention: rotary + append + attention in one call, the
+    query-tile kernel rotating its Q rows as it loads them (q_rot receives
+    only the decode tokens' rows; out and the cache equal the two-call path's)."""
+    _check(lib().fg_rotary_kv_attention(cache.handle, batch.handle, _dev_ptr(q, "q"), _dev_ptr(k, "k"),
+                                        _dev_ptr(v, "v"), _dev_ptr(q_rot, "q_rot"), _dev_ptr(out, "out"),
+                                        int(n_q_heads), float(rope_theta), float(softmax_scale),
+                                        int(sliding_window), _stream_ptr(stream)),
+           "fg_rotary_kv_attention")
 
 
 def ragged_attention_noalloc(cache: KVCache, batch: RaggedBatch, q_rot, out, n_q_heads: int,
