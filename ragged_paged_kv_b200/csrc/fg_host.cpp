@@ -1194,13 +1194,15 @@ extern "C" fg_status fg_qkv_rotary_kv_append(fg_kv_cache* c, const fg_ragged_bat
   if (st) return st;
   const int d = c->head_dim;
   const uint64_t n_out = (uint64_t)(n_q_heads + 2 * c->n_kv_heads) * d;
+  // the persistent 128 x 256 tile form when the output width allows it
+  const bool persistent = n_out % 256 == 0;
   CUtensorMap tm_x, tm_w;
   if (!make_rows_map(&tm_x, x, (uint64_t)hidden, (uint64_t)b->n_tokens, 128) ||
-      !make_rows_map(&tm_w, w_qkv, (uint64_t)hidden, n_out, (uint32_t)d))
+      !make_rows_map(&tm_w, w_qkv, (uint64_t)hidden, n_out, persistent ? 256u : (uint32_t)d))
     return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed for x or w_qkv");
   cudaError_t e = fg::launch_qkv_rotary_append(&tm_x, &tm_w, cache_view(c), b->view,
                                                static_cast<__nv_bfloat16*>(q_rot), c->rope, n_q_heads, hidden,
-                                               static_cast<cudaStream_t>(stream));
+                                               static_cast<cudaStream_t>(stream), persistent);
   if (e != cudaSuccess) return cuda_fail(e, "qkv_rotary_append launch");
   return FG_OK;
 }
@@ -1220,7 +1222,7 @@ extern "C" fg_status fg_output_projection(const fg_ragged_batch* b, const void* 
   if (!attn_out || !w_o || !y) return fail(FG_ERR_INVALID_ARG, "NULL tensor pointer");
   if (!aligned16(attn_out) || !aligned16(w_o) || !aligned16(y))
     return fail(FG_ERR_INVALID_ARG, "attn_out, w_o and y must be 16-byte aligned");
-  const uint32_t n_tile = out_features % 128 == 0 ? 128 : 64;
+  const uint32_t n_tile = out_features % 256 == 0 ? 256 : out_features % 128 == 0 ? 128 : 64;
   CUtensorMap tm_x, tm_w;
   if (!make_rows_map(&tm_x, attn_out, (uint64_t)in_features, (uint64_t)b->n_tokens, 128) ||
       !make_rows_map(&tm_w, w_o, (uint64_t)in_features, (uint64_t)out_features, n_tile))

@@ -124,14 +124,18 @@ cudaError_t launch_attention_decode_tc(const void* tm_q1, const void* tm_kv, con
                                        int sm_tc_end, const int* tc_counter, int n_tc, bool pdl,
                                        cudaStream_t stream);
 
+// persistent: the 128 x 256 tile form (one CTA per SM, two TMEM
+// accumulators; the output width (n_q_heads + 2 Hkv) d a multiple of 256,
+// tm_w with 64 x 256 boxes); otherwise one 128-token x d tile per CTA
+// (tm_w with 64 x d boxes). tm_x has 64 x 128 boxes.
 cudaError_t launch_qkv_rotary_append(const void* tm_x, const void* tm_w, const CacheView& cache,
                                      const BatchView& batch, __nv_bfloat16* q_rot, const double2* rope,
-                                     int n_q_heads, int hidden, cudaStream_t stream);
+                                     int n_q_heads, int hidden, cudaStream_t stream, bool persistent);
 
 // y[T][n_out] = x[T][k_len] w[n_out][k_len]^T in bf16 with fp32 accumulation
 // (the layer's output projection); T = batch.n_tokens, n_tile (64 or 128)
-// output features per CTA, tm_x / tm_w 2-D maps with 64 x 128 and
-// 64 x n_tile boxes.
+// output features per CTA, or 256: the persistent 128 x 256 tile form;
+// tm_x / tm_w 2-D maps with 64 x 128 and 64 x n_tile boxes.
 cudaError_t launch_linear_bf16(const void* tm_x, const void* tm_w, const BatchView& batch, __nv_bfloat16* y,
                                int k_len, int n_out, int n_tile, cudaStream_t stream);
 

@@ -337,7 +337,7 @@ def near(got_bits, ref_bits, scale, what, acc=0.0):
     assert np.mean(got_bits != ref_bits) < 0.01, f"{what}: {np.mean(got_bits != ref_bits):.3%} words differ"
 
 
-@pytest.mark.parametrize("which", ["mha_d64", "gqa_d128"])
+@pytest.mark.parametrize("which", ["mha_d64", "gqa_d128", "gqa_d64_one_tile_per_head"])
 def test_fused_qkv_projection_rotary_append(which):
     """fg_qkv_rotary_kv_append: the projection x W^T fused with rotary and the
     append. Against the oracle's exact projection (rounded once to bf16) the
@@ -350,6 +350,10 @@ def test_fused_qkv_projection_rotary_append(which):
         w = W._make("qkv_mha_d64", 4, 4, 64, 16, [0, 1, 2, 3], [40, 1, 1, 22], [0, 37, 5, 10], seed=21,
                     budget=64)
         hidden = 256
+    elif which == "gqa_d64_one_tile_per_head":
+        # (4 + 2) x 64 = 384 outputs, not a multiple of 256: the one-tile-per-head form
+        w = W._make("qkv_gqa_d64", 4, 1, 64, 32, [0, 1, 2], [150, 1, 9], [0, 300, 41], seed=24, budget=160)
+        hidden = 192
     else:
         w = W._make("qkv_gqa_d128", 8, 2, 128, 64, [0, 1, 2], [300, 1, 17], [0, 700, 70], seed=22, budget=318)
         hidden = 512
@@ -502,18 +506,20 @@ def test_fused_qkv_projection_at_llama7b_width():
     _free(cache, batch)
 
 
-@pytest.mark.parametrize("which", ["tiny_n64", "ragged_n128", "llama7b_width"])
+@pytest.mark.parametrize("which", ["tiny_n64", "ragged_n128", "ragged_n384", "llama7b_width"])
 def test_output_projection(which):
     """fg_output_projection: y = o W_o^T against the oracle's exactly summed
     linear layer rounded once to bf16. The GPU's fp32 sums may round a value
     to the neighbouring bf16, so every word is within the rounding of both
     sides plus the fp32 accumulation bound, and almost all are identical.
-    The cases cover 64- and 128-wide output tiles and a token count with a
+    The cases cover 64- and 128-wide output tiles, the persistent 256-wide
+    form (output widths that are multiples of 256) and a token count with a
     ragged last 128-row tile."""
     from oracle import linear
     # (tokens as q_lens of a few sequences, in_features, out_features)
     shapes = {"tiny_n64": ([40, 1, 1, 22], 256, 192),
               "ragged_n128": ([300, 1, 17], 512, 256),
+              "ragged_n384": ([300, 1, 17], 512, 384),
               "llama7b_width": ([517, 1, 1, 11], 4096, 4096)}
     q_lens, k_in, n_out = shapes[which]
     S = len(q_lens)
