@@ -534,8 +534,9 @@ def make_workload(config, compact_pool=False, local_rank=0, gpu=True):
     return w
 
 
-# gates of the five configurations (the benchmark's table): the dominant
-# kernel's fraction of its roofline
+# the gates of the measured configurations: the dominant kernel's fraction of
+# its roofline (HBM bandwidth for the decode-heavy batches, the bf16 tensor
+# peak for the long-prompt batch)
 GATES = {2: ("hbm", 0.70), 3: ("hbm", 0.70), 4: ("hbm", 0.70), 5: ("tensor", 0.50)}
 
 
