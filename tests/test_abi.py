@@ -141,3 +141,22 @@ def test_prepare_rotary_rejects_bad_arguments():
     assert fg.STATUS[L.fg_kv_cache_prepare_rotary(h, 10000.0, -1)] == "FG_ERR_INVALID_ARG"
     assert fg.STATUS[L.fg_kv_cache_prepare_rotary(None, 10000.0, 100)] == "FG_ERR_INVALID_ARG"
     L.fg_kv_cache_destroy(h)
+
+
+def test_one_call_pass_rejects_bad_arguments():
+    """fg_rotary_kv_attention checks its handles and arguments before any
+    device work: a batch not put against this cache, NULL handles, a
+    non-positive rope_theta or softmax_scale, a negative window."""
+    h = _external()
+    b = fg.RaggedBatch(max_tokens=8, max_seqs=2, max_blocks_per_seq=2)
+    L = fg.lib()
+    d = ctypes.c_void_p(FAKE_DEV)
+    z = ctypes.c_void_p(0)
+
+    def call(cache, batch, theta=10000.0, scale=0.125, window=0, heads=2):
+        return fg.STATUS[L.fg_rotary_kv_attention(cache, batch, d, d, d, d, d, heads, theta, scale, window, z)]
+
+    assert call(h, b.handle) == "FG_ERR_INVALID_ARG"     # no put against this cache yet
+    assert call(None, b.handle) == "FG_ERR_INVALID_ARG"
+    assert call(h, None) == "FG_ERR_INVALID_ARG"
+    L.fg_kv_cache_destroy(h)

@@ -101,3 +101,30 @@ def test_fused_pass_shape_sweep(B, d, Hq, Hkv, window):
     w = W._make(f"sweep_B{B}_d{d}_g{Hq // Hkv}_w{window}", Hq, Hkv, d, B, list(range(7)),
                 q_lens, ctx_lens, seed=int(rng.integers(1 << 30)), budget=sum(q_lens), window=window)
     _check(w)
+
+
+def test_fused_pass_rejects_bad_arguments():
+    """After a valid put: q_rot equal to q, a non-positive rope_theta or
+    softmax_scale, a negative window and a misaligned pointer are rejected
+    before any launch, and the cache is untouched."""
+    w = W.config1()
+    cache = fg.KVCache(w.block_size, w.n_blocks, w.n_kv_heads, w.head_dim)
+    fixtures.fill(cache.tensor)
+    before = to_bits(cache.tensor)
+    batch = fg.RaggedBatch(w.n_tokens, w.n_seqs, w.block_tables.shape[1])
+    batch.put(cache, w.seq_ids, w.q_lens, w.ctx_lens, w.block_tables)
+    q, k, v = fixtures.qkv_device(w)
+    q_rot, out = torch.empty_like(q), torch.empty_like(q)
+    bad = [dict(q_rot=q), dict(rope_theta=0.0), dict(softmax_scale=0.0), dict(sliding_window=-1),
+           dict(out=out.view(-1)[1:])]
+    for b in bad:
+        args = dict(q_rot=q_rot, out=out, rope_theta=w.rope_theta, softmax_scale=w.softmax_scale, sliding_window=0)
+        args.update(b)
+        with pytest.raises(fg.FgError) as e:
+            fg.rotary_kv_attention(cache, batch, q, k, v, args["q_rot"], args["out"], w.n_q_heads,
+                                   args["rope_theta"], args["softmax_scale"], args["sliding_window"])
+        assert e.value.name == "FG_ERR_INVALID_ARG", (b, e.value.name)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_bits(cache.tensor), before)
+    cache.close()
+    batch.close()
