@@ -544,7 +544,7 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
   }
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (!b->derr) {
-    b->dmeta_words = 3 * (size_t)b->max_seqs + 2 + (size_t)b->max_tokens +
+    b->dmeta_words = 3 * (size_t)b->max_seqs + 2 + 3 * (size_t)b->max_tokens +
                      (size_t)b->max_seqs * b->max_blocks_per_seq;
     FG_CUDA(cudaGetDevice(&b->device));
     if (!b->copy) {
@@ -562,8 +562,10 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
   int half = 0;
   st = b->meta.begin(b->dmeta_words * 4, true, strm, b->copy, &half);
   if (st) return st;
-  // pack: cu_q[S+1] ctx[S] bt_off[S+1] tok_seq[T] bt[nblk]
-  const size_t words = 3 * (size_t)S + 2 + (size_t)T + (size_t)nblk;
+  // pack: cu_q[S+1] ctx[S] bt_off[S+1] tok_seq[T] tok_pos[T] tok_blk[T] bt[nblk]
+  // (each row's position and block resolved here, so the append's producer
+  // reads them with one load instead of a chain of dependent ones)
+  const size_t words = 3 * (size_t)S + 2 + 3 * (size_t)T + (size_t)nblk;
   void* hp = nullptr;
   int slot = 0;
   const double t_w = now_us();
@@ -575,7 +577,9 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
   int32_t* cx = cu + S + 1;
   int32_t* bo = cx + S;
   int32_t* ts = bo + S + 1;
-  int32_t* bb = ts + T;
+  int32_t* tp = ts + T;
+  int32_t* tb = tp + T;
+  int32_t* bb = tb + T;
   cu[0] = 0;
   bo[0] = 0;
   const int64_t B = c->block_size;
@@ -585,7 +589,13 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
     const int64_t nb = ((int64_t)cl[s] + ql[s] + B - 1) / B;
     bo[s + 1] = bo[s] + (int32_t)nb;
     std::memcpy(bb + bo[s], bt + (int64_t)s * stride, (size_t)nb * 4);
-    for (int32_t j = 0; j < ql[s]; ++j) ts[cu[s] + j] = s;
+    const int32_t* row = bt + (int64_t)s * stride;
+    for (int32_t j = 0; j < ql[s]; ++j) {
+      const int32_t pos = cl[s] + j;
+      ts[cu[s] + j] = s;
+      tp[cu[s] + j] = pos;
+      tb[cu[s] + j] = row[pos / B];
+    }
   }
   int32_t* d = static_cast<int32_t*>(b->meta.buf[half]);
   st = b->meta_stage.copy(slot, d, words * 4, b->copy);
@@ -597,7 +607,9 @@ extern "C" fg_status fg_ragged_batch_put(fg_ragged_batch* b, const fg_kv_cache* 
   b->view.ctx = d + S + 1;
   b->view.bt_off = d + 2 * S + 1;
   b->view.tok_seq = d + 3 * S + 2;
-  b->view.bt = d + 3 * S + 2 + T;
+  b->view.tok_pos = d + 3 * S + 2 + T;
+  b->view.tok_blk = d + 3 * S + 2 + 2 * T;
+  b->view.bt = d + 3 * S + 2 + 3 * T;
   b->view.n_seqs = S;
   b->view.n_tokens = (int32_t)T;
   b->view.err = b->derr;

@@ -75,6 +75,8 @@ struct BatchView {
   const int32_t* bt_off;   // [S + 1] CSR offsets into bt
   const int32_t* bt;       // physical block ids, logical order per sequence
   const int32_t* tok_seq;  // [T] sequence index of each batch row
+  const int32_t* tok_pos;  // [T] absolute position of each batch row (ctx + index in its sequence)
+  const int32_t* tok_blk;  // [T] physical block holding that position's cache slot
   int32_t n_seqs;
   int32_t n_tokens;
   int32_t* err;            // device error word

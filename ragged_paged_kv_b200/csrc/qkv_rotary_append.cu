@@ -113,14 +113,13 @@ __device__ __forceinline__ void epilogue_row(const QkvArgs& a, uint32_t (&acc)[D
 #pragma unroll
     for (int e = 0; e < D; ++e) acc[e] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(acc[e])));
     const int Hkv = a.cache.n_kv_heads;
-    const int s = a.batch.tok_seq[t];
-    const int p = a.batch.ctx[s] + (t - a.batch.cu_q[s]);
+    const int p = a.batch.tok_pos[t];
     __nv_bfloat16* dst = nullptr;
     if (head < a.Hq) {
       dst = a.q_rot + ((int64_t)t * a.Hq + head) * D;
     } else {
       const int lb = p / a.cache.block_size;
-      const int32_t blk = a.batch.bt[a.batch.bt_off[s] + lb];
+      const int32_t blk = a.batch.tok_blk[t];
       if (blk >= 0 && blk < a.cache.n_blocks) {
         const int kv = head < a.Hq + Hkv ? 0 : 1;
         dst = a.cache.base +

@@ -45,9 +45,10 @@ struct RotCfg {
 
 // A unit is (token, chunk of 32 heads of the concatenated q | k | v rows).
 // Warp 4 is the producer. For each batch of 32 of the CTA's units
-// (blockIdx.x, + gridDim.x, ...) its lane j resolves unit j's sequence,
-// position and cache block (a chain of dependent metadata loads; the 32
-// chains run at once) into a shared batch table; lane 0 then, stage by
+// (blockIdx.x, + gridDim.x, ...) its lane j reads unit j's position and
+// cache block (two independent loads of per-row arrays the batch put
+// resolved on the host; the 32 lanes' loads run at once) into a shared batch
+// table; lane 0 then, stage by
 // stage, writes a unit's metadata into the stage and pulls its rows (each of
 // q, k and v a contiguous run of whole heads) and the position's rotary row
 // with 1-D bulk copies on the stage's mbarrier. Warps 0-3 rotate from shared
@@ -92,9 +93,7 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
         if (u < n_units) {
           const int t = u / chunks;
           const int h0 = (u - t * chunks) * kChunkHeads;
-          const int s = batch.tok_seq[t];
-          const int pos = batch.ctx[s] + (t - batch.cu_q[s]);
-          const int lb = pos / cache.block_size;
+          const int pos = batch.tok_pos[t];
           m.t = t;
           m.h0 = h0;
           m.h1 = min(h0 + kChunkHeads, Hq + 2 * Hkv);
@@ -103,12 +102,13 @@ __global__ void __launch_bounds__(kConsumers + 32, kCtasPerSm) rotary_append_ker
           // it serves, the plan's rule with skip_tc_q = the largest group the
           // tensor-core decode kernel takes): the unit keeps its K and V
           if (skip_tc_q > 0 && h0 < Hq) {
+            const int s = batch.tok_seq[t];
             const int qn = batch.cu_q[s + 1] - batch.cu_q[s];
             const int grp = Hq / Hkv;
             if (!(qn == 1 && ((D == 128 && grp <= skip_tc_q) || grp == 1))) m.h0 = min(Hq, m.h1);
           }
-          m.blk = batch.bt[batch.bt_off[s] + lb];
-          m.slot = pos - lb * cache.block_size;
+          m.blk = batch.tok_blk[t];
+          m.slot = pos - (pos / cache.block_size) * cache.block_size;
           m.pos = pos;
         }
         batch_meta[lane] = m;
