@@ -618,7 +618,9 @@ def run_fg(args, w, rank, ws, local_rank):
     d1.record(pipe.up)
     d1.synchronize()
     both_ms = d0.elapsed_time(d1) / args.steps
-    meta_bytes = 4 * (3 * w.n_seqs + 2 + w.n_tokens +
+    # the put's metadata upload: cu_q, ctx, bt_off, the per-row sequence,
+    # position and block, and the compact block tables (int32)
+    meta_bytes = 4 * (3 * w.n_seqs + 2 + 3 * w.n_tokens +
                       sum(w.blocks_used(s) for s in range(w.n_seqs)))
     h2d = sum(t.numel() * 2 for t in host_in.values()) + meta_bytes
     d2h = host_out.numel() * 2
