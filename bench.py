@@ -139,9 +139,10 @@ def load_peaks():
 class ClockSampler:
     """SM clock and clock-event reasons during the timed region, read-only.
 
-    Polls NVML every 2 ms (the timed region of a short run lasts only a few
-    milliseconds; nvidia-smi could sample it once at best), and falls back to
-    nvidia-smi every 200 ms where NVML is unavailable."""
+    Polls NVML every 0.5 ms (the timed region of a short run lasts only a few
+    milliseconds; nvidia-smi could sample it once at best; the NVML calls go
+    through ctypes, which lets the enqueuing thread run meanwhile), and falls
+    back to nvidia-smi every 200 ms where NVML is unavailable."""
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4))
@@ -168,7 +169,7 @@ class ClockSampler:
             except Exception:
                 h = pynvml.nvmlDeviceGetHandleByIndex(index)
             self._nvml = (pynvml, h, pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
-            self.source = "nvml, 2 ms"
+            self.source = "nvml, 0.5 ms"
         except Exception:
             self._nvml = None
 
@@ -182,7 +183,7 @@ class ClockSampler:
                     self.samples.append((float(sm), float(mx), [n for n, m in self.REASONS if bits & m]))
                 except Exception:
                     pass
-                self._stop.wait(0.002)
+                self._stop.wait(0.0005)
             return
         self.source = "nvidia-smi, 200 ms"
         while not self._stop.is_set():
