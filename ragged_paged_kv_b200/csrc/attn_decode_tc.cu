@@ -186,6 +186,8 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
       const int B = a.cache.block_size;
       const int BR = B < 64 ? B : 64;
       const int Hkv = a.cache.n_kv_heads;
+      // each key's K and V is read by one unit only: evict those lines first
+      const uint64_t l2_once = ptx::l2_evict_first_policy();
       int gt = 0, un = 0;
       for (;; ++un) {
         int u = -1;
@@ -227,8 +229,8 @@ __global__ void __launch_bounds__(192, 2) attn_decode_tc_kernel(const __grid_con
                 continue;
               }
               const int r0 = (int)((((int64_t)blk * 2 + kv) * Hkv + h) * B + (pos - lb * B));
-              ptx::tma_load_2d(dst + (pos - k0) * 128, &tm_kv, 0, r0, &slot_full[slot]);
-              ptx::tma_load_2d(dst + C::BK * 128 + (pos - k0) * 128, &tm_kv, 64, r0, &slot_full[slot]);
+              ptx::tma_load_2d_hint(dst + (pos - k0) * 128, &tm_kv, 0, r0, &slot_full[slot], l2_once);
+              ptx::tma_load_2d_hint(dst + C::BK * 128 + (pos - k0) * 128, &tm_kv, 64, r0, &slot_full[slot], l2_once);
             }
           }
         }
