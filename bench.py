@@ -116,7 +116,7 @@ def algorithmic_work(w):
 # (null in the line) where no capture was taken or the kernel has changed
 # since. Summaries with the commands are in profiles/.
 NCU_TRAFFIC = {
-    2: {"decode": 1264466944, "tc": 53071360},
+    2: {"decode": 1263240448, "tc": 53071360},
     5: {"tc": 416548608},
 }
 
