@@ -405,9 +405,12 @@ __global__ void __launch_bounds__(384, 1) attn_tc_kernel(const __grid_constant__
             }
             const int row = (int)((((int64_t)blk * 2 + kv) * Hkv + x.h) * B + (pos - (pos / B) * B));
 #pragma unroll
+            // the unit order puts CTAs that read the same kv head's keys side
+            // by side, so these lines are read again soon: keep them in L2
+            // ahead of the lines streamed once (Q, the decode kernel's K/V)
             for (int dh = 0; dh < C::DH; ++dh)
-              ptx::tma_load_2d(ring + st * C::kKVBytes + dh * C::BN * 128 + (pos - k0) * 128, &tm_kv, dh * 64,
-                               row, &full[st]);
+              ptx::tma_load_2d_hint(ring + st * C::kKVBytes + dh * C::BN * 128 + (pos - k0) * 128, &tm_kv,
+                                    dh * 64, row, &full[st], ptx::l2_evict_last_policy());
           }
 #pragma unroll
           for (int j = 0; j < kMaxBoxes; ++j) cur[j] = nxt[j];
